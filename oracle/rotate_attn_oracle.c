@@ -1,0 +1,390 @@
+/*
+ * CPU oracle for the RotateAttention INT4 attention forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check
+ * and the benchmark's CPU-baseline leg may load this library.  It is a plain,
+ * slow, obviously-correct restatement of what the method computes; it shares
+ * no code, header, table or constant generator with the CUDA library.
+ *
+ * Source: "RotateAttention: RoPE-Aware Rotation and Range Rectification for
+ * INT4 Quantized Attention in Video Generation" (arXiv 2607.02584), as
+ * summarised on its review page:
+ *   - 3D RoPE splits head_dim into frame / height / width segments
+ *     (core claim; axiom ledger; Fig. 2 caption);
+ *   - RoPE-aware rotation: block-diagonal 2x2 orthogonal blocks, either on
+ *     adjacent dims (Interleaved, mergeable into RoPE) or pairing a dim with
+ *     its counterpart in the other half of its segment (Half)
+ *     (Fig. 3 caption; "What carries the argument");
+ *   - blocks initialised to the 2x2 Hadamard H2 (free-parameter ledger);
+ *   - INT4 FlashAttention with online softmax (abstract);
+ *   - range-optimised P quantisation: P = exp(QK^T - max) in [0,1] mapped to
+ *     [-8,7] with fixed scale 15 and zero-point -8 (Sec. 4.2; ledger);
+ *   - the V column-sum term that corrects the zero-point in P.V.
+ * Where the pages are silent the plainest reading is taken; each such reading
+ * is marked READING below.
+ *
+ * Precision: every step that decides an integer (a Q/K/V code, a P code)
+ * is taken in IEEE fp32 with no FMA contraction (build with
+ * -ffp-contract=off), because that is the precision the CUDA path decides in;
+ * integer products are exact (int32/int64); the running accumulators of the
+ * online softmax are float64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef _Float16 f16;
+
+/* The oracle's own description of one problem. */
+typedef struct {
+    int B, H, d;          /* batch, heads, head_dim (128) */
+    int F, Hh, W;         /* latent video grid, frame-major */
+    int n_text;           /* text tokens appended after the video tokens */
+    int split[3];         /* RoPE segment sizes (frame, height, width) */
+    double theta;         /* RoPE base */
+    int rot;              /* 0 = no rotation, 1 = Interleaved, 2 = Half */
+} orc_problem;
+
+enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2 };
+enum { QK_BLOCK = 64, KV_TILE = 128 };
+
+int orc_seq_len(const orc_problem *p) { return p->F * p->Hh * p->W + p->n_text; }
+
+/* Padded length: a whole number of 128-token tiles. */
+int orc_seq_pad(const orc_problem *p) { return (orc_seq_len(p) + KV_TILE - 1) / KV_TILE * KV_TILE; }
+
+/* Token n -> axis positions (frame, row, column).  Video tokens are laid out
+ * frame-major (f slowest, w fastest); appended text tokens sit at position 0
+ * on every axis, i.e. RoPE leaves them unchanged.  READING: the pages give
+ * neither the token order nor the text-token convention. */
+void orc_token_pos(const orc_problem *p, int n, int pos[3])
+{
+    int nv = p->F * p->Hh * p->W;
+    if (n >= nv) { pos[0] = pos[1] = pos[2] = 0; return; }
+    pos[0] = n / (p->Hh * p->W);
+    pos[1] = (n / p->W) % p->Hh;
+    pos[2] = n % p->W;
+}
+
+/* RoPE angle for axis segment s, axis position pos, pair j (dims o_s+2j and
+ * o_s+2j+1 of the segment): pos * theta^(-2j/d_s), in float64. */
+double orc_rope_angle(const orc_problem *p, int s, int pos, int j)
+{
+    double w = pow(p->theta, -(double)(2 * j) / (double)p->split[s]);
+    return (double)pos * w;
+}
+
+/* The fp32 coefficients the prologue uses, each rounded once from float64:
+ * (cos a, sin a) for RoPE alone, and (alpha, beta) for RoPE followed by the
+ * 2x2 Hadamard H2 on the same adjacent pair (the Interleaved rotation merged
+ * into RoPE): H2 * [[c,-s],[s,c]] = [[alpha, beta],[beta, -alpha]] with
+ * alpha = (c+s)/sqrt2, beta = (c-s)/sqrt2. */
+void orc_rope_coef(const orc_problem *p, int s, int pos, int j,
+                   float *c, float *sn, float *alpha, float *beta)
+{
+    double a = orc_rope_angle(p, s, pos, j);
+    double ca = cos(a), sa = sin(a);
+    *c = (float)ca;
+    *sn = (float)sa;
+    *alpha = (float)((ca + sa) * M_SQRT1_2);
+    *beta = (float)((ca - sa) * M_SQRT1_2);
+}
+
+/* RoPE (no rotation) of one token in fp32: each adjacent pair (x0, x1) of a
+ * segment becomes (c x0 - s x1, s x0 + c x1). */
+static void rope_row(const orc_problem *p, int n, const f16 *x, float *y)
+{
+    int pos[3];
+    orc_token_pos(p, n, pos);
+    int o = 0;
+    for (int s = 0; s < 3; ++s) {
+        for (int j = 0; j < p->split[s] / 2; ++j) {
+            float c, sn, al, be;
+            orc_rope_coef(p, s, pos[s], j, &c, &sn, &al, &be);
+            float x0 = (float)x[o + 2 * j], x1 = (float)x[o + 2 * j + 1];
+            float a0 = c * x0, a1 = sn * x1;
+            float b0 = sn * x0, b1 = c * x1;
+            y[o + 2 * j] = a0 - a1;
+            y[o + 2 * j + 1] = b0 + b1;
+        }
+        o += p->split[s];
+    }
+}
+
+/* RoPE then the RoPE-aware rotation of one token (Q or K), fp32.
+ *  - none:        z = RoPE(x)
+ *  - Interleaved: H2 after RoPE on each adjacent pair, with the merged
+ *                 (alpha, beta) coefficients: z0 = alpha x0 + beta x1,
+ *                 z1 = beta x0 - alpha x1
+ *  - Half:        z = RoPE(x), then in each segment dim i and dim i + d_s/2
+ *                 (a, b) -> ((a+b)/sqrt2, (a-b)/sqrt2).
+ * READING: rotation after RoPE (either order leaves QK^T unchanged); H2 is
+ * the default block (free-parameter ledger). */
+void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
+{
+    if (p->rot == ORC_ROT_INTERLEAVED) {
+        int pos[3];
+        orc_token_pos(p, n, pos);
+        int o = 0;
+        for (int s = 0; s < 3; ++s) {
+            for (int j = 0; j < p->split[s] / 2; ++j) {
+                float c, sn, al, be;
+                orc_rope_coef(p, s, pos[s], j, &c, &sn, &al, &be);
+                float x0 = (float)x[o + 2 * j], x1 = (float)x[o + 2 * j + 1];
+                float a0 = al * x0, a1 = be * x1;
+                float b0 = be * x0, b1 = al * x1;
+                z[o + 2 * j] = a0 + a1;
+                z[o + 2 * j + 1] = b0 - b1;
+            }
+            o += p->split[s];
+        }
+        return;
+    }
+    float y[512];
+    rope_row(p, n, x, y);
+    if (p->rot == ORC_ROT_NONE) {
+        memcpy(z, y, sizeof(float) * p->d);
+        return;
+    }
+    const float r = (float)M_SQRT1_2;
+    int o = 0;
+    for (int s = 0; s < 3; ++s) {
+        int h = p->split[s] / 2;
+        for (int i = 0; i < h; ++i) {
+            float a = y[o + i], b = y[o + i + h];
+            float sum = a + b, dif = a - b;
+            z[o + i] = sum * r;
+            z[o + i + h] = dif * r;
+        }
+        o += p->split[s];
+    }
+}
+
+/* RoPE only, rounded to fp16 (RNE): the FP16 path's Q/K after RoPE. */
+void orc_rope_fp16_head(const orc_problem *p, const f16 *x, f16 *y)
+{
+    int N = orc_seq_len(p), d = p->d;
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        float t[512];
+        rope_row(p, n, x + (size_t)n * d, t);
+        for (int c = 0; c < d; ++c) y[(size_t)n * d + c] = (f16)t[c];
+    }
+}
+
+/* Symmetric INT4 code of v with scale s: clamp(rne(v / s), -7, 7), 0 if s == 0. */
+static int8_t int4_code(float v, float s)
+{
+    if (s == 0.0f) return 0;
+    float q = nearbyintf(v / s);
+    if (q > 7.0f) q = 7.0f;
+    if (q < -7.0f) q = -7.0f;
+    return (int8_t)q;
+}
+
+/* Q or K of one head: RoPE + rotation, then per 64-token block one scale
+ * amax/7 over all 64 x d values and codes rne(z/scale) in [-7, 7].
+ * codes: [N_pad][d], padded tokens 0; scales: [N_pad/64], padded blocks 0.
+ * READING: the 64-token block matches the FlashAttention block size used by
+ * block-wise attention quantisation; V is handled by orc_quantize_v_head. */
+void orc_quantize_qk_head(const orc_problem *p, const f16 *x, int8_t *codes, float *scales)
+{
+    int N = orc_seq_len(p), Np = orc_seq_pad(p), d = p->d;
+    float *z = (float *)malloc(sizeof(float) * (size_t)N * d);
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) orc_rotate_row(p, n, x + (size_t)n * d, z + (size_t)n * d);
+    memset(codes, 0, (size_t)Np * d);
+    for (int g = 0; g < Np / QK_BLOCK; ++g) {
+        int n0 = g * QK_BLOCK, n1 = n0 + QK_BLOCK < N ? n0 + QK_BLOCK : N;
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float a = fabsf(z[(size_t)n * d + c]);
+                if (a > amax) amax = a;
+            }
+        float s = amax / 7.0f;
+        scales[g] = s;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c)
+                codes[(size_t)n * d + c] = int4_code(z[(size_t)n * d + c], s);
+    }
+    free(z);
+}
+
+/* V of one head: one symmetric INT4 scale per channel over all N tokens
+ * (amax_c / 7), codes in [-7, 7], and the per-64-token-block column sums of
+ * the codes used by the zero-point correction.  No transform is applied to V:
+ * the paper's Hadamard on V is fused offline into the model weights.
+ * codes: [N_pad][d]; sv: [d]; colsum: [N_pad/64][d].
+ * READING: the pages fix no granularity for V; per-channel over the whole
+ * sequence keeps the scale constant along the P.V contraction. */
+void orc_quantize_v_head(const orc_problem *p, const f16 *v, int8_t *codes, float *sv, int32_t *colsum)
+{
+    int N = orc_seq_len(p), Np = orc_seq_pad(p), d = p->d;
+    for (int c = 0; c < d; ++c) {
+        float amax = 0.0f;
+        for (int n = 0; n < N; ++n) {
+            float a = fabsf((float)v[(size_t)n * d + c]);
+            if (a > amax) amax = a;
+        }
+        sv[c] = amax / 7.0f;
+    }
+    memset(codes, 0, (size_t)Np * d);
+    memset(colsum, 0, sizeof(int32_t) * (size_t)(Np / QK_BLOCK) * d);
+    for (int n = 0; n < N; ++n)
+        for (int c = 0; c < d; ++c) {
+            int8_t q = int4_code((float)v[(size_t)n * d + c], sv[c]);
+            codes[(size_t)n * d + c] = q;
+            colsum[(size_t)(n / QK_BLOCK) * d + c] += q;
+        }
+}
+
+/* Range-optimised P code: P in [0,1] -> rne(15 P) - 8 in [-8, 7]
+ * (fixed scale 15, zero-point -8; Sec. 4.2). */
+int orc_p_code(float P) { return (int)nearbyintf(15.0f * P) - 8; }
+
+/* One query row i of the INT4 attention (one head), T_kv = `tile` keys per
+ * step of the online softmax (128 for the method as built).
+ *
+ * Per tile j (keys [n0, n1)):
+ *   S[n]  = sum_c q_code[i,c] k_code[n,c]                         (int32)
+ *   s[n]  = S[n] * (s_Q[i/64] * s_K[n/64]) * (1/sqrt d)            (fp32)
+ *   m_j   = max(m_{j-1}, max_n s[n])                               (fp32)
+ *   P[n]  = exp(s[n] - m_j);  code[n] = rne(15 P) - 8              (fp32)
+ *   PV[c] = sum_n code[n] v_code[n,c] + 8 colsum_j[c]              (int64)
+ *   L     = sum_n (code[n] + 8)                                    (int64)
+ *   acc   = acc * exp(m_{j-1} - m_j) + PV;  l = l * exp(..) + L    (float64)
+ * O[i,c] = acc[c] * s_V[c] / l, rounded to fp16; the common 1/15 cancels.
+ * READINGS: the standard 1/sqrt(d) softmax scale applies to the dequantised
+ * logits; the normaliser uses the dequantised codes (keeps O a convex
+ * combination of dequantised V rows); P is quantised against the running max.
+ *
+ * quant_p = 0 replaces the P code by the exact P (float64) and drops the
+ * zero-point, for checking the loop against two-pass softmax attention.
+ * Optional outputs: o64 [d] (float64 before the fp16 rounding); for tile
+ * index dbg_tile >= 0, dbg_S [tile] and dbg_P [tile] (S and P codes of that
+ * tile, -128 where the key is past N).
+ * colsum: [N_pad/64][d] per-64-block column sums of the V codes. */
+void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
+                       const int8_t *qc, const float *qs, const int8_t *kc, const float *ks,
+                       const int8_t *vc, const float *sv, const int32_t *colsum,
+                       f16 *o, double *o64, int dbg_tile, int32_t *dbg_S, int8_t *dbg_P)
+{
+    int N = orc_seq_len(p), d = p->d;
+    const float inv_sqrt_d = (float)(1.0 / sqrt((double)d));
+    float m = -INFINITY;
+    double *acc = (double *)calloc((size_t)d, sizeof(double));
+    double l = 0.0;
+    int32_t *S = (int32_t *)malloc(sizeof(int32_t) * (size_t)tile);
+    float *sl = (float *)malloc(sizeof(float) * (size_t)tile);
+    double *pv = (double *)malloc(sizeof(double) * (size_t)d);
+    const int8_t *qrow = qc + (size_t)i * d;
+    for (int j = 0, n0 = 0; n0 < N; ++j, n0 += tile) {
+        int n1 = n0 + tile < N ? n0 + tile : N;
+        float tmax = -INFINITY;
+        for (int n = n0; n < n1; ++n) {
+            int32_t acc_s = 0;
+            for (int c = 0; c < d; ++c) acc_s += (int32_t)qrow[c] * (int32_t)kc[(size_t)n * d + c];
+            S[n - n0] = acc_s;
+            float sc = qs[i / QK_BLOCK] * ks[n / QK_BLOCK];
+            float t = (float)acc_s * sc;
+            float s = t * inv_sqrt_d;
+            sl[n - n0] = s;
+            if (s > tmax) tmax = s;
+        }
+        float m_new = m > tmax ? m : tmax;
+        double L = 0.0;
+        for (int c = 0; c < d; ++c) pv[c] = 0.0;
+        if (quant_p) {
+            int64_t pvi[512] = {0};
+            int64_t Li = 0;
+            for (int n = n0; n < n1; ++n) {
+                float P = expf(sl[n - n0] - m_new);
+                int code = orc_p_code(P);
+                Li += code + 8;
+                for (int c = 0; c < d; ++c) pvi[c] += (int64_t)code * vc[(size_t)n * d + c];
+                if (j == dbg_tile && dbg_P) dbg_P[n - n0] = (int8_t)code;
+            }
+            /* zero-point correction: + 8 * sum over the tile's keys of the V codes */
+            for (int g = n0 / QK_BLOCK; g * QK_BLOCK < n1; ++g)
+                for (int c = 0; c < d; ++c) pvi[c] += 8 * (int64_t)colsum[(size_t)g * d + c];
+            for (int c = 0; c < d; ++c) pv[c] = (double)pvi[c];
+            L = (double)Li;
+        } else {
+            for (int n = n0; n < n1; ++n) {
+                double P = exp((double)sl[n - n0] - (double)m_new);
+                L += P;
+                for (int c = 0; c < d; ++c) pv[c] += P * (double)vc[(size_t)n * d + c];
+            }
+        }
+        if (j == dbg_tile) {
+            for (int n = 0; n < tile; ++n) {
+                if (dbg_S) dbg_S[n] = n0 + n < n1 ? S[n] : 0;
+                if (dbg_P && n0 + n >= n1) dbg_P[n] = -128;
+            }
+        }
+        double alpha = (j == 0) ? 0.0 : exp((double)m - (double)m_new);
+        for (int c = 0; c < d; ++c) acc[c] = acc[c] * alpha + pv[c];
+        l = l * alpha + L;
+        m = m_new;
+    }
+    for (int c = 0; c < d; ++c) {
+        double val = acc[c] * (double)sv[c] / l;
+        if (o64) o64[c] = val;
+        if (o) o[c] = (f16)val;
+    }
+    free(acc); free(S); free(sl); free(pv);
+}
+
+/* Rows `rows[0..nrows)` of one head; out: [nrows][d] fp16, out64 optional. */
+void orc_attention_rows(const orc_problem *p, const int64_t *rows, int nrows, int tile, int quant_p,
+                        const int8_t *qc, const float *qs, const int8_t *kc, const float *ks,
+                        const int8_t *vc, const float *sv, const int32_t *colsum,
+                        f16 *out, double *out64)
+{
+    int d = p->d;
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int r = 0; r < nrows; ++r)
+        orc_attention_row(p, (int)rows[r], tile, quant_p, qc, qs, kc, ks, vc, sv, colsum,
+                          out ? out + (size_t)r * d : NULL, out64 ? out64 + (size_t)r * d : NULL,
+                          -1, NULL, NULL);
+}
+
+/* Float64 softmax attention of one head on given (already position-encoded)
+ * fp32 or fp16-valued rows: O[i] = sum_n softmax_n(q_i.k_n / sqrt d) v_n.
+ * Used for the unquantised diagnostic and as the FP16 path's oracle. */
+void orc_softmax_attention_rows(const orc_problem *p, const int64_t *rows, int nrows,
+                                const double *q, const double *k, const double *v, double *out)
+{
+    int N = orc_seq_len(p), d = p->d;
+    double scale = 1.0 / sqrt((double)d);
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int r = 0; r < nrows; ++r) {
+        const double *qi = q + (size_t)rows[r] * d;
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        double mx = -INFINITY;
+        for (int n = 0; n < N; ++n) {
+            double t = 0.0;
+            for (int c = 0; c < d; ++c) t += qi[c] * k[(size_t)n * d + c];
+            s[n] = t * scale;
+            if (s[n] > mx) mx = s[n];
+        }
+        double den = 0.0;
+        for (int n = 0; n < N; ++n) { s[n] = exp(s[n] - mx); den += s[n]; }
+        double *o = out + (size_t)r * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        for (int n = 0; n < N; ++n)
+            for (int c = 0; c < d; ++c) o[c] += s[n] * v[(size_t)n * d + c];
+        for (int c = 0; c < d; ++c) o[c] /= den;
+        free(s);
+    }
+}
+
+/* Rotated fp32 rows of one head (RoPE + rotation, before quantisation). */
+void orc_rotate_head(const orc_problem *p, const f16 *x, float *z)
+{
+    int N = orc_seq_len(p), d = p->d;
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) orc_rotate_row(p, n, x + (size_t)n * d, z + (size_t)n * d);
+}

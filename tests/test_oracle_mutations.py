@@ -1,0 +1,44 @@
+"""The pins must catch plausible mistakes: each case below plants one slip in
+a copy of the oracle's C source (on the CPU), builds it, and requires the pin
+suite to fail against it."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+from oracle import oracle as O
+
+MUTANTS = {
+    "drop_zero_point": ("pvi[c] += 8 * (int64_t)colsum", "pvi[c] += 0 * (int64_t)colsum"),
+    "swap_scale_index": ("qs[i / QK_BLOCK] * ks[n / QK_BLOCK]", "qs[n / QK_BLOCK] * ks[i / QK_BLOCK]"),
+    "rope_sign": ("y[o + 2 * j] = a0 - a1;", "y[o + 2 * j] = a0 + a1;"),
+    "interleaved_sign": ("z[o + 2 * j + 1] = b0 - b1;", "z[o + 2 * j + 1] = b0 + b1;"),
+    "half_partner": ("float a = y[o + i], b = y[o + i + h];", "float a = y[o + i], b = y[o + h - 1 - i];"),
+    "p_scale_16": ("nearbyintf(15.0f * P) - 8", "nearbyintf(16.0f * P) - 8"),
+    "global_not_running_max": ("float m_new = m > tmax ? m : tmax;", "float m_new = tmax > m ? tmax : tmax;"),
+    "rescale_sign": ("exp((double)m - (double)m_new)", "exp((double)m_new - (double)m)"),
+    "qk_scale_8": ("float s = amax / 7.0f;", "float s = amax / 8.0f;"),
+    "rope_freq": ("-(double)(2 * j) / (double)p->split[s]", "-(double)(j) / (double)p->split[s]"),
+    "token_order": ("pos[1] = (n / p->W) % p->Hh;", "pos[1] = (n / p->Hh) % p->W;"),
+    "v_scale_per_tensor": ("sv[c] = amax / 7.0f;", "sv[c] = (amax > sv[0] ? amax : sv[0]) / 7.0f;"),
+    "softmax_scale": ("(float)(1.0 / sqrt((double)d))", "(float)(1.0 / (double)d)"),
+    "normaliser_exact_p": ("Li += code + 8;", "Li += 15;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(O.SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    msrc = tmp_path / "mutant.c"
+    msrc.write_text(src.replace(old, new))
+    mlib = str(tmp_path / "libmutant.so")
+    O.compile_oracle(str(msrc), mlib)
+    env = dict(os.environ, RA_ORACLE_LIB=mlib)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(root, "tests", "test_oracle_pins.py")],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
