@@ -1,0 +1,329 @@
+#!/usr/bin/env python
+"""Benchmark of the RotateAttention INT4 attention forward on B200.
+
+One step = one pass of the hot path over the Wan2.2-shaped workload
+(B=1, H=40, N=21*45*80=75,600, d=128): ra_rotate_quantize_qkv followed by
+ra_int4_attention_fwd, inputs resident in HBM.  Metric: INT4 attention TOPS
+= 4*N^2*d*H / time.  Prints one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--config wan|hunyuan|half|tiny] [--schedule]
+
+--impl reference times the CPU oracle (the only reference this method has:
+the paper released no kernels) on a bounded sample of the same workload.
+Multi-GPU: replicas only (the path has no exchange step); each rank runs the
+same workload on its own GPU and the value is the sum over ranks, timed as
+the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_quantized_attention_b200 import synth  # noqa: E402
+from int4_quantized_attention_b200.schedule import BENCH_SCHEDULE  # noqa: E402
+
+METRIC = "INT4 attention TOPS (4*N^2*d*H/time) and fraction of B200 INT8 tensor peak"
+KERNELS_PER_STEP = 4      # qk_quant, v_amax, v_quant, int4_attn
+# Nominal dense tensor rates: int8 (= fp8) is twice bf16/fp16 on B200.
+INT8_PER_BF16 = 2.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(cfg, budget_s: float = 12.0, max_rows: int = 4096):
+    """Time the oracle on a bounded sample: the prologue of head 0 and the
+    INT4 attention of query rows of head 0, in batches until the budget."""
+    from oracle import oracle as O
+    O.build_oracle()
+    q, k, v = synth.make_qkv(cfg, heads=1)
+    t0 = time.perf_counter()
+    qz = O.quantize_head(cfg, q[0, 0], k[0, 0], v[0, 0])
+    t_pro = time.perf_counter() - t0
+    rng = np.random.default_rng(5)
+    rows_done, t_att = 0, 0.0
+    while t_att < budget_s and rows_done < max_rows:
+        rows = rng.choice(cfg.N, 64, replace=False).astype(np.int64)
+        t0 = time.perf_counter()
+        O.attention_rows(cfg, qz, rows=rows)
+        t_att += time.perf_counter() - t0
+        rows_done += len(rows)
+    ops = 4.0 * rows_done * cfg.N * cfg.d
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return dict(value=ops / t_att / 1e12, unit="TOPS", cores=cores, kind="oracle",
+                sample=f"{cfg.name}: INT4 attention of {rows_done} query rows of head 0 "
+                       f"({rows_done * cfg.N} row-key pairs, {t_att:.1f} s); head-0 prologue "
+                       f"{t_pro:.2f} s not counted in the TOPS",
+                seconds=t_att)
+
+
+def reference_arm(args, cfg, rank):
+    if rank != 0:
+        return
+    cb = cpu_oracle_sample(cfg, budget_s=max(3.0, min(20.0, 4.0 * args.steps)))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int32", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
+                       "grid": [cfg.F, cfg.Hh, cfg.W], "n_text": cfg.n_text, "split": list(cfg.split),
+                       "rotation": cfg.rot},
+            "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": {"value": cb["value"], "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def event_time(fn, iters, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(iters):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / iters
+
+
+def our_arm(args, cfg, rank, world):
+    import torch
+    import torch.distributed as dist
+    from int4_quantized_attention_b200 import api, build
+
+    build.build()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+
+    q, k, v = synth.make_qkv(cfg)
+    qd, kd, vd = (torch.from_numpy(t).to(dev) for t in (q, k, v))
+    ra = api.RotateAttention(cfg, dev, fp16_path=True)
+    out = torch.empty_like(qd)
+
+    def step():
+        ra.rotate_quantize(qd, kd, vd)
+        ra.int4_attention(out)
+
+    for _ in range(args.warmup):
+        step()
+    ra.check()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms_step = event_time(step, args.steps, stream)
+        # the dominant kernel alone, on the same stream (inputs > L2 between launches)
+        ms_attn = event_time(lambda: ra.int4_attention(out), args.steps, stream)
+        ms_pro = event_time(lambda: ra.rotate_quantize(qd, kd, vd), max(args.steps, 10), stream)
+    ra.check()
+    torch.cuda.synchronize()
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+        dist.barrier()
+
+    # FP16 path on the same workload (a few calls)
+    ms_f16 = event_time(lambda: ra.fp16_attention(qd, kd, vd, out), max(2, args.steps // 3), stream)
+    ra.check()
+
+    # end to end through the public API with host buffers
+    qh, kh, vh = (torch.from_numpy(t).pin_memory() for t in (q, k, v))
+    oh = torch.empty(out.shape, dtype=torch.float16).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(out, non_blocking=True)
+
+    e2e_step()
+    ms_e2e = event_time(e2e_step, max(2, args.steps // 2), stream)
+    ra.check()
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    sched = None
+    if args.schedule:
+        sched = run_schedule(ra, qd, kd, vd, out, stream)
+
+    if rank != 0:
+        return
+    ops = cfg.ops
+    tops = world * ops / (ms_step * 1e-3) / 1e12
+    attn_tops = ops / (ms_attn * 1e-3) / 1e12
+    peak_int8 = peaks["bf16_sus"] * INT8_PER_BF16
+    Np = ra.N_pad
+    BH = cfg.B * cfg.H
+    pro_bytes = (3 * BH * cfg.N * cfg.d * 2            # read q, k, v
+                 + BH * cfg.N * cfg.d * 2              # second read of v (after its amax)
+                 + 3 * BH * Np * cfg.d // 2            # packed INT4 writes
+                 + BH * (Np // 64) * cfg.d * 4)        # V column sums
+    cpu = cpu_oracle_sample(cfg, budget_s=12.0) if not args.no_cpu_baseline else None
+    line = {
+        "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8xs8->s32 (INT4 codes), fp32 softmax", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
+                   "grid": [cfg.F, cfg.Hh, cfg.W], "n_text": cfg.n_text, "split": list(cfg.split),
+                   "rotation": cfg.rot, "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "l2": "inputs larger than L2 (q,k,v 2.3 GB; packed K/V 0.39 GB per pass)"},
+        "roofline": {"kernel": "int4_attn_kernel", "bound": "tensor", "achieved": attn_tops,
+                     "peak": peak_int8, "unit": "TOPS", "frac": attn_tops / peak_int8, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sus']} TF/s x 2 (int8:bf16 "
+                                    f"nominal ratio); burst-based peak {peaks['bf16'] * INT8_PER_BF16:.0f}"},
+        "int4_attention_ms": ms_attn,
+        "prologue": {"ms": ms_pro, "algorithmic_bytes": pro_bytes,
+                     "achieved_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
+                     "frac_hbm": pro_bytes / (ms_pro * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "fp16_path": {"ms": ms_f16, "tflops": ops / (ms_f16 * 1e-3) / 1e12,
+                      "frac_bf16_peak": ops / (ms_f16 * 1e-3) / 1e12 / peaks["bf16_sus"],
+                      "int4_step_speedup": ms_f16 / ms_step},
+        "e2e": {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
+                "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "gpu": torch.cuda.get_device_name(dev),
+    }
+    if sched is not None:
+        line["schedule"] = sched
+    print(json.dumps(line), flush=True)
+
+
+def run_schedule(ra, qd, kd, vd, out, stream):
+    """Mixed-precision schedule: per (step, block) the FP16 or the INT4 path,
+    each call timed with events; compared with all-FP16."""
+    import torch
+    kinds = [kind for _, _, kind in BENCH_SCHEDULE.calls()]
+    per = {"int4": [], "fp16": []}
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in kinds]
+    torch.cuda.synchronize()
+    for kind, (a, b) in zip(kinds, evs):
+        a.record(stream)
+        ra.forward(qd, kd, vd, path=kind, out=out)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for kind, (a, b) in zip(kinds, evs):
+        per[kind].append(a.elapsed_time(b))
+    mixed = sum(per["int4"]) + sum(per["fp16"])
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in kinds]
+    for a, b in evs2:
+        a.record(stream)
+        ra.forward(qd, kd, vd, path="fp16", out=out)
+        b.record(stream)
+    torch.cuda.synchronize()
+    all16 = sum(a.elapsed_time(b) for a, b in evs2)
+    ra.check()
+    return {"calls": len(kinds), "int4_fraction": BENCH_SCHEDULE.int4_fraction,
+            "int4_ms_per_call": statistics.median(per["int4"]), "fp16_ms_per_call": statistics.median(per["fp16"]),
+            "mixed_total_ms": mixed, "all_fp16_total_ms": all16, "speedup_vs_all_fp16": all16 / mixed}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="wan", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--schedule", action="store_true", help="also run the 400-call mixed schedule")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = synth.CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, cfg, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        our_arm(args, cfg, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

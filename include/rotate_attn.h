@@ -1,0 +1,171 @@
+/*
+ * rotate_attn.h -- C ABI of the RotateAttention INT4 attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "RotateAttention: RoPE-Aware Rotation and Range Rectification for
+ * INT4 Quantized Attention in Video Generation" (arXiv 2607.02584), as
+ * described on its review page (pith summary, core claim, "What carries the
+ * argument", free-parameter ledger, abstract, Fig. 2 and Fig. 3 captions).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers, 16-byte aligned, row-major and contiguous.
+ *     fp16 tensors are [B][H][N][d] with d = 128.
+ *   - The caller owns all memory.  The library allocates and frees nothing on
+ *     any call; it only reads and writes the buffers it is given.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns without synchronising, except ra_check_device_error.
+ *   - Errors are status codes; nothing throws or aborts across the ABI.
+ *     Argument errors are found on the host before any launch and nothing is
+ *     enqueued then.  ra_last_error_detail() gives a one-line reason for the
+ *     last non-OK status of the calling thread.
+ *   - Device-side faults are not raised as CUDA errors: every bounded wait
+ *     and every self-check in the kernels records a code in the workspace's
+ *     error word; ra_check_device_error() reads and clears it.
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef ROTATE_ATTN_H
+#define ROTATE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RA_OK = 0,
+    RA_ERR_INVALID_ARG = 1,     /* bad shape, split, mode, null or misaligned pointer */
+    RA_ERR_UNSUPPORTED = 2,     /* valid in principle, not built (e.g. d != 128) */
+    RA_ERR_WORKSPACE = 3,       /* workspace too small or not prepared for this problem */
+    RA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+    RA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out */
+    RA_ERR_DEVICE_BOUNDS = 6    /* a device-side self-check found a bad index */
+} ra_status;
+
+typedef enum {
+    RA_ROT_NONE = 0,            /* RoPE only */
+    RA_ROT_INTERLEAVED = 1,     /* H2 on adjacent dims, merged into RoPE (Fig. 3) */
+    RA_ROT_HALF = 2             /* H2 on (i, i + d_s/2) in each segment (Fig. 3) */
+} ra_rot_mode;
+
+/* One attention problem.  Tokens: N = F*Hh*W video tokens in frame-major
+ * order (frame slowest, column fastest) followed by n_text text tokens, which
+ * get no RoPE but do get the rotation.  head_dim d is split into three RoPE
+ * segments split[0..2] (frame, height, width; each even, sum = d); pair j of
+ * segment s (dims o_s+2j, o_s+2j+1) turns by pos_s * theta^(-2j/split[s]). */
+typedef struct {
+    int B, H, d;
+    int F, Hh, W, n_text;
+    int split[3];
+    double theta;               /* RoPE base, e.g. 10000.0 */
+    int rot;                    /* ra_rot_mode */
+} ra_problem;
+
+/* Quantised Q, K, V as produced by ra_rotate_quantize_qkv (device memory).
+ * N_pad = N rounded up to a multiple of 128; padded tokens hold code 0.
+ *   q4, k4 : uint8 [B][H][N_pad][64]  two INT4 codes per byte, channel 2c in
+ *            the low nibble and 2c+1 in the high nibble, two's complement,
+ *            codes in [-7, 7]
+ *   v4t    : uint8 [B][H][128][N_pad/2]  V transposed (channel-major), token
+ *            2t in the low nibble and 2t+1 in the high nibble
+ *   sq, sk : float [B][H][N_pad/64]   one scale per 64-token block (amax/7)
+ *   sv     : float [B][H][128]        one scale per channel over all N tokens
+ *   vsum   : int32 [B][H][N_pad/64][128]  per-64-token-block column sums of
+ *            the V codes (the zero-point correction term of P.V) */
+typedef struct {
+    uint8_t *q4, *k4, *v4t;
+    float *sq, *sk, *sv;
+    int32_t *vsum;
+} ra_qkv4;
+
+typedef void *ra_stream;        /* cudaStream_t */
+
+/* Sequence length N and padded length N_pad of a problem (-1 if invalid). */
+int ra_seq_len(const ra_problem *p);
+int ra_seq_pad(const ra_problem *p);
+
+/* Checks a problem: B, H >= 1; d == 128 (else RA_ERR_UNSUPPORTED); grid
+ * sizes >= 0 with N >= 1; split entries even, positive, summing to d;
+ * rot in ra_rot_mode; theta > 0; every tensor under 2^31 elements per head. */
+ra_status ra_validate(const ra_problem *p);
+
+/* Bytes of one device buffer that holds all of ra_qkv4 (sub-buffers aligned
+ * to 256 bytes), and the binding of such a buffer into an ra_qkv4. */
+size_t ra_qkv4_bytes(const ra_problem *p);
+ra_status ra_qkv4_bind(const ra_problem *p, void *base, size_t bytes, ra_qkv4 *out);
+
+/* Workspace: error word, RoPE/rotation tables, V channel-amax scratch and,
+ * when with_fp16_path != 0, the FP16 path's position-encoded Q, K and
+ * transposed V (3 * B*H*N_pad*128 fp16).  Device memory owned by the caller. */
+size_t ra_workspace_bytes(const ra_problem *p, int with_fp16_path);
+
+/* Builds the RoPE/rotation coefficient tables on the host (float64 libm,
+ * each coefficient rounded once to fp32), copies them into the workspace
+ * with cudaMemcpyAsync on `stream`, clears the error word and records the
+ * problem's signature.  Call once per (problem, workspace) before the other
+ * calls; they check the signature on the device and report
+ * RA_ERR_WORKSPACE through ra_check_device_error when it does not match. */
+ra_status ra_prepare(const ra_problem *p, void *workspace, size_t workspace_bytes, ra_stream stream);
+
+/* Fused prologue: 3D RoPE and the RoPE-aware rotation of Q and K, per
+ * 64-token-block symmetric INT4 quantisation of Q and K, per-channel
+ * symmetric INT4 quantisation of V with transposed packing and column sums.
+ * q, k, v: fp16 [B][H][N][128]; out: bound by ra_qkv4_bind.
+ * ("What carries the argument"; Fig. 3 caption; free-parameter ledger.) */
+ra_status ra_rotate_quantize_qkv(const ra_problem *p, const void *q, const void *k, const void *v,
+                                 const ra_qkv4 *out, void *workspace, size_t workspace_bytes,
+                                 ra_stream stream);
+
+/* INT4 attention forward: S = Q K^T on INT8 tensor cores (INT4 codes widened
+ * to INT8), online softmax over 128-key tiles, P = exp(s - m) quantised to
+ * rne(15 P) - 8, P.V with the zero-point correction, fp16 output.
+ * in: from ra_rotate_quantize_qkv; o: fp16 [B][H][N][128].
+ * (Abstract; Sec. 4.2 as summarised in the referee report and ledger.) */
+ra_status ra_int4_attention_fwd(const ra_problem *p, const ra_qkv4 *in, void *o,
+                                void *workspace, size_t workspace_bytes, ra_stream stream);
+
+/* FP16 path (the pages' mixed-precision fallback, abstract and Sec. 5.1):
+ * 3D RoPE in fp32 rounded to fp16 (no rotation: an orthogonal rotation does
+ * not change full-precision attention), then FlashAttention with fp32
+ * accumulation.  q, k, v, o: fp16 [B][H][N][128].  Needs a workspace sized
+ * with with_fp16_path != 0. */
+ra_status ra_fp16_attention_fwd(const ra_problem *p, const void *q, const void *k, const void *v,
+                                void *o, void *workspace, size_t workspace_bytes, ra_stream stream);
+
+/* Synchronises `stream`, reads and clears the workspace's error word.
+ * Returns RA_OK, RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS or
+ * RA_ERR_WORKSPACE (signature mismatch), or RA_ERR_CUDA. */
+ra_status ra_check_device_error(void *workspace, ra_stream stream);
+
+const char *ra_status_string(ra_status s);
+const char *ra_last_error_detail(void);
+
+/* ---- test hooks ------------------------------------------------------- */
+
+/* Number of floats of the coefficient table and the table itself, as
+ * ra_prepare uploads it: for segment s, position pos in [0, P_s) with
+ * P = (F, Hh, W), pair j: {cos, sin, alpha, beta} at
+ * 4 * (off_s + pos * split[s]/2 + j), off_0 = 0, off_{s+1} = off_s + P_s*split[s]/2. */
+size_t ra_tables_floats(const ra_problem *p);
+ra_status ra_build_tables_host(const ra_problem *p, float *out, size_t n_floats);
+
+/* Runs the INT4 attention for one (b*H + h, 128-row query tile) through the
+ * same kernel and records, for KV tile kv_tile, the int32 S tile
+ * (s_out: device int32 [128][128], S[row][key], keys past N = 0) and the P
+ * codes (p_out: device int8 [128][128], code in [-8, 7], -128 past N). */
+ra_status ra_debug_int4_tile(const ra_problem *p, const ra_qkv4 *in, int bh, int q_tile, int kv_tile,
+                             int32_t *s_out, int8_t *p_out, void *workspace, size_t workspace_bytes,
+                             ra_stream stream);
+
+/* Sets the iteration limit of every bounded device-side wait (0 restores the
+ * default); a test sets 1 and runs ra_debug_timeout_probe, whose kernel waits
+ * on a barrier that nothing arms and must return RA_ERR_DEVICE_TIMEOUT via
+ * ra_check_device_error. */
+void ra_debug_set_wait_limit(uint32_t iterations);
+ra_status ra_debug_timeout_probe(void *workspace, size_t workspace_bytes, ra_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ROTATE_ATTN_H */

@@ -1,0 +1,360 @@
+// ra_api.cu -- host side of the C ABI declared in include/rotate_attn.h:
+// argument validation, RoPE/rotation coefficient tables, workspace layout,
+// error reporting and kernel launches.  No allocation anywhere: every buffer
+// is the caller's.
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "ra_internal.h"
+
+namespace {
+
+thread_local char g_detail[256] = "";
+std::atomic<uint32_t> g_wait_limit{0};
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;   // polls of mbarrier.try_wait (about a second)
+
+ra_status fail(ra_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ra_status fail(ra_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+ra_status cuda_fail(cudaError_t e, const char* what) {
+  cudaGetLastError();   // clear the sticky-free error so later calls start clean
+  return fail(RA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint64_t fnv1a(const void* data, size_t n, uint64_t h = 1469598103934665603ull) {
+  const unsigned char* b = static_cast<const unsigned char*>(data);
+  for (size_t i = 0; i < n; ++i) h = (h ^ b[i]) * 1099511628211ull;
+  return h;
+}
+
+// Validates and derives the kernel-side sizes.
+ra_status derive(const ra_problem* p, ra::Prob* out) {
+  if (p == nullptr) return fail(RA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->B < 1 || p->H < 1) return fail(RA_ERR_INVALID_ARG, "B and H must be >= 1 (got %d, %d)", p->B, p->H);
+  if (p->d != ra::D) return fail(RA_ERR_UNSUPPORTED, "head_dim %d: only 128 is built", p->d);
+  if (p->F < 0 || p->Hh < 0 || p->W < 0 || p->n_text < 0)
+    return fail(RA_ERR_INVALID_ARG, "negative grid or text size");
+  const long long nv = (long long)p->F * p->Hh * p->W;
+  const long long N = nv + p->n_text;
+  if (N < 1) return fail(RA_ERR_INVALID_ARG, "empty sequence (N = 0)");
+  const bool any_zero = p->F == 0 || p->Hh == 0 || p->W == 0;
+  const bool all_zero = p->F == 0 && p->Hh == 0 && p->W == 0;
+  if (any_zero && !all_zero) return fail(RA_ERR_INVALID_ARG, "video grid with a zero axis (use 0x0x0 for text only)");
+  int sum = 0;
+  for (int s = 0; s < 3; ++s) {
+    if (p->split[s] <= 0 || (p->split[s] & 1))
+      return fail(RA_ERR_INVALID_ARG, "RoPE segment %d size %d must be even and positive", s, p->split[s]);
+    sum += p->split[s];
+  }
+  if (sum != p->d) return fail(RA_ERR_INVALID_ARG, "RoPE split sums to %d, head_dim is %d", sum, p->d);
+  if (p->rot != RA_ROT_NONE && p->rot != RA_ROT_INTERLEAVED && p->rot != RA_ROT_HALF)
+    return fail(RA_ERR_INVALID_ARG, "rotation mode %d unknown", p->rot);
+  if (!(p->theta > 0.0) || !std::isfinite(p->theta)) return fail(RA_ERR_INVALID_ARG, "RoPE base must be > 0");
+  const long long Np = (N + ra::TILE - 1) / ra::TILE * ra::TILE;
+  if (Np * ra::D >= (1ll << 31)) return fail(RA_ERR_UNSUPPORTED, "sequence too long: %lld tokens", N);
+  if ((long long)p->B * p->H > 65535) return fail(RA_ERR_UNSUPPORTED, "B*H > 65535");
+  if (out) {
+    ra::Prob& P = *out;
+    P.B = p->B;
+    P.H = p->H;
+    P.BH = p->B * p->H;
+    P.N = (int)N;
+    P.N_pad = (int)Np;
+    P.n_video = (int)nv;
+    P.F = p->F;
+    P.Hh = p->Hh;
+    P.W = p->W;
+    P.rot = p->rot;
+    const int npos[3] = {p->F > 0 ? p->F : 1, p->Hh > 0 ? p->Hh : 1, p->W > 0 ? p->W : 1};
+    int off = 0, toff = 0;
+    for (int s = 0; s < 3; ++s) {
+      P.split[s] = p->split[s];
+      P.off[s] = off;
+      off += p->split[s];
+      P.npos[s] = npos[s];
+      P.tab_off[s] = toff;
+      toff += npos[s] * (p->split[s] / 2);
+    }
+    P.n_tab = toff;
+    uint64_t h = fnv1a(&p->B, sizeof(int) * 7);
+    h = fnv1a(p->split, sizeof(p->split), h);
+    h = fnv1a(&p->theta, sizeof(double), h);
+    h = fnv1a(&p->rot, sizeof(int), h);
+    P.signature = h | 1ull;   // never 0, so a zeroed workspace never matches
+  }
+  return RA_OK;
+}
+
+// Coefficients {cos a, sin a, (cos a + sin a)/sqrt2, (cos a - sin a)/sqrt2}
+// per (segment, position, pair), a = pos * theta^(-2j/d_s), each computed in
+// float64 and rounded once to fp32.
+void build_tables(const ra_problem* p, const ra::Prob& P, float* out) {
+  for (int s = 0; s < 3; ++s) {
+    const int half = p->split[s] / 2;
+    for (int pos = 0; pos < P.npos[s]; ++pos)
+      for (int j = 0; j < half; ++j) {
+        const double w = std::pow(p->theta, -(double)(2 * j) / (double)p->split[s]);
+        const double a = (double)pos * w;
+        const double ca = std::cos(a), sa = std::sin(a);
+        float* e = out + 4 * ((size_t)P.tab_off[s] + (size_t)pos * half + j);
+        e[0] = (float)ca;
+        e[1] = (float)sa;
+        e[2] = (float)((ca + sa) * M_SQRT1_2);
+        e[3] = (float)((ca - sa) * M_SQRT1_2);
+      }
+  }
+}
+
+struct QkvLayout {
+  size_t q4, k4, v4t, sq, sk, sv, vsum, total;
+};
+
+QkvLayout qkv_layout(const ra::Prob& P) {
+  QkvLayout L;
+  size_t o = 0;
+  const size_t packed = (size_t)P.BH * P.N_pad * (ra::D / 2);
+  L.q4 = o;
+  o = ra::align256(o + packed);
+  L.k4 = o;
+  o = ra::align256(o + packed);
+  L.v4t = o;
+  o = ra::align256(o + packed);
+  L.sq = o;
+  o = ra::align256(o + sizeof(float) * (size_t)P.BH * (P.N_pad / ra::QK_BLOCK));
+  L.sk = o;
+  o = ra::align256(o + sizeof(float) * (size_t)P.BH * (P.N_pad / ra::QK_BLOCK));
+  L.sv = o;
+  o = ra::align256(o + sizeof(float) * (size_t)P.BH * ra::D);
+  L.vsum = o;
+  o = ra::align256(o + sizeof(int32_t) * (size_t)P.BH * (P.N_pad / ra::QK_BLOCK) * ra::D);
+  L.total = o;
+  return L;
+}
+
+ra_status check_ws(const ra::Prob& P, const void* ws, size_t bytes, bool fp16) {
+  if (!aligned16(ws)) return fail(RA_ERR_INVALID_ARG, "workspace pointer NULL or not 16-byte aligned");
+  const ra::WsLayout L = ra::ws_layout(P);
+  const size_t need = fp16 ? L.total_fp16 : L.base_bytes;
+  if (bytes < need) return fail(RA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", bytes, need);
+  return RA_OK;
+}
+
+ra_status check_qkv4(const ra_qkv4* t) {
+  if (t == nullptr) return fail(RA_ERR_INVALID_ARG, "ra_qkv4 is NULL");
+  if (!aligned16(t->q4) || !aligned16(t->k4) || !aligned16(t->v4t) || !aligned16(t->sq) || !aligned16(t->sk) ||
+      !aligned16(t->sv) || !aligned16(t->vsum))
+    return fail(RA_ERR_INVALID_ARG, "an ra_qkv4 pointer is NULL or not 16-byte aligned");
+  return RA_OK;
+}
+
+}  // namespace
+
+namespace ra {
+uint32_t wait_limit() {
+  const uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
+  return v ? v : kDefaultWaitLimit;
+}
+}  // namespace ra
+
+extern "C" {
+
+int ra_seq_len(const ra_problem* p) {
+  ra::Prob P;
+  return derive(p, &P) == RA_OK ? P.N : -1;
+}
+
+int ra_seq_pad(const ra_problem* p) {
+  ra::Prob P;
+  return derive(p, &P) == RA_OK ? P.N_pad : -1;
+}
+
+ra_status ra_validate(const ra_problem* p) { return derive(p, nullptr); }
+
+size_t ra_qkv4_bytes(const ra_problem* p) {
+  ra::Prob P;
+  if (derive(p, &P) != RA_OK) return 0;
+  return qkv_layout(P).total;
+}
+
+ra_status ra_qkv4_bind(const ra_problem* p, void* base, size_t bytes, ra_qkv4* out) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if (out == nullptr) return fail(RA_ERR_INVALID_ARG, "output ra_qkv4 is NULL");
+  if (base == nullptr || (reinterpret_cast<uintptr_t>(base) & 255u))
+    return fail(RA_ERR_INVALID_ARG, "qkv4 buffer NULL or not 256-byte aligned");
+  const QkvLayout L = qkv_layout(P);
+  if (bytes < L.total) return fail(RA_ERR_INVALID_ARG, "qkv4 buffer has %zu bytes, needs %zu", bytes, L.total);
+  char* b = static_cast<char*>(base);
+  out->q4 = reinterpret_cast<uint8_t*>(b + L.q4);
+  out->k4 = reinterpret_cast<uint8_t*>(b + L.k4);
+  out->v4t = reinterpret_cast<uint8_t*>(b + L.v4t);
+  out->sq = reinterpret_cast<float*>(b + L.sq);
+  out->sk = reinterpret_cast<float*>(b + L.sk);
+  out->sv = reinterpret_cast<float*>(b + L.sv);
+  out->vsum = reinterpret_cast<int32_t*>(b + L.vsum);
+  return RA_OK;
+}
+
+size_t ra_workspace_bytes(const ra_problem* p, int with_fp16_path) {
+  ra::Prob P;
+  if (derive(p, &P) != RA_OK) return 0;
+  const ra::WsLayout L = ra::ws_layout(P);
+  return with_fp16_path ? L.total_fp16 : L.base_bytes;
+}
+
+size_t ra_tables_floats(const ra_problem* p) {
+  ra::Prob P;
+  if (derive(p, &P) != RA_OK) return 0;
+  return 4 * (size_t)P.n_tab;
+}
+
+ra_status ra_build_tables_host(const ra_problem* p, float* out, size_t n_floats) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if (out == nullptr || n_floats < 4 * (size_t)P.n_tab)
+    return fail(RA_ERR_INVALID_ARG, "table buffer NULL or smaller than %zu floats", 4 * (size_t)P.n_tab);
+  build_tables(p, P, out);
+  return RA_OK;
+}
+
+ra_status ra_prepare(const ra_problem* p, void* ws, size_t ws_bytes, ra_stream stream) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ra::WsLayout L = ra::ws_layout(P);
+  std::vector<float> tab(4 * (size_t)P.n_tab);
+  build_tables(p, P, tab.data());
+  ra::WsHeader hdr{};
+  hdr.signature = P.signature;
+  char* base = static_cast<char*>(ws);
+  // Pageable source: the runtime stages both copies before returning.
+  cudaError_t e = cudaMemcpyAsync(base + L.tables, tab.data(), sizeof(float) * tab.size(), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  e = cudaMemcpyAsync(base, &hdr, sizeof(hdr), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "header upload");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "prepare");
+  return RA_OK;
+}
+
+ra_status ra_rotate_quantize_qkv(const ra_problem* p, const void* q, const void* k, const void* v,
+                                 const ra_qkv4* out, void* ws, size_t ws_bytes, ra_stream stream) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v))
+    return fail(RA_ERR_INVALID_ARG, "q, k or v NULL or not 16-byte aligned");
+  if ((st = check_qkv4(out)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  cudaError_t e = ra::launch_prologue(P, static_cast<const __half*>(q), static_cast<const __half*>(k),
+                                      static_cast<const __half*>(v), out->q4, out->k4, out->v4t, out->sq, out->sk,
+                                      out->sv, out->vsum, ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "prologue launch");
+}
+
+ra_status ra_int4_attention_fwd(const ra_problem* p, const ra_qkv4* in, void* o, void* ws, size_t ws_bytes,
+                                ra_stream stream) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if ((st = check_qkv4(in)) != RA_OK) return st;
+  if (!aligned16(o)) return fail(RA_ERR_INVALID_ARG, "output NULL or not 16-byte aligned");
+  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  cudaError_t e = ra::launch_int4_attention(P, in->q4, in->k4, in->v4t, in->sq, in->sk, in->sv,
+                                            static_cast<__half*>(o), ws, -1, -1, -1, nullptr, nullptr,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "int4 attention launch");
+}
+
+ra_status ra_fp16_attention_fwd(const ra_problem* p, const void* q, const void* k, const void* v, void* o, void* ws,
+                                size_t ws_bytes, ra_stream stream) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(RA_ERR_INVALID_ARG, "q, k, v or o NULL or not 16-byte aligned");
+  if ((st = check_ws(P, ws, ws_bytes, true)) != RA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = ra::launch_fp16_prologue(P, static_cast<const __half*>(q), static_cast<const __half*>(k),
+                                           static_cast<const __half*>(v), ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fp16 prologue launch");
+  e = ra::launch_fp16_attention(P, static_cast<__half*>(o), ws, s);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "fp16 attention launch");
+}
+
+ra_status ra_check_device_error(void* ws, ra_stream stream) {
+  if (!aligned16(ws)) return fail(RA_ERR_INVALID_ARG, "workspace pointer NULL or not 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  ra::DeviceErr err{};
+  e = cudaMemcpy(&err, ws, sizeof(err), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "error word read");
+  if (err.word == 0) return RA_OK;
+  e = cudaMemset(ws, 0, sizeof(err));
+  if (e != cudaSuccess) return cuda_fail(e, "error word clear");
+  if (err.word & ra::DEVERR_WORKSPACE)
+    return fail(RA_ERR_WORKSPACE, "workspace not prepared for this problem (site 0x%x)", err.site);
+  if (err.word & ra::DEVERR_BOUNDS) return fail(RA_ERR_DEVICE_BOUNDS, "device bounds check (site 0x%x)", err.site);
+  return fail(RA_ERR_DEVICE_TIMEOUT, "bounded device wait ran out (site 0x%x)", err.site);
+}
+
+const char* ra_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "ok";
+    case RA_ERR_INVALID_ARG: return "invalid argument";
+    case RA_ERR_UNSUPPORTED: return "unsupported";
+    case RA_ERR_WORKSPACE: return "workspace too small or not prepared";
+    case RA_ERR_CUDA: return "CUDA error";
+    case RA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case RA_ERR_DEVICE_BOUNDS: return "device bounds check failed";
+  }
+  return "unknown status";
+}
+
+const char* ra_last_error_detail(void) { return g_detail; }
+
+ra_status ra_debug_int4_tile(const ra_problem* p, const ra_qkv4* in, int bh, int q_tile, int kv_tile,
+                             int32_t* s_out, int8_t* p_out, void* ws, size_t ws_bytes, ra_stream stream) {
+  ra::Prob P;
+  ra_status st = derive(p, &P);
+  if (st != RA_OK) return st;
+  if ((st = check_qkv4(in)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  if (bh < 0 || bh >= P.BH || q_tile < 0 || q_tile >= P.N_pad / ra::TILE || kv_tile < 0 ||
+      kv_tile >= P.N_pad / ra::TILE)
+    return fail(RA_ERR_INVALID_ARG, "debug tile index out of range");
+  if (!aligned16(s_out) || !aligned16(p_out)) return fail(RA_ERR_INVALID_ARG, "debug outputs NULL or misaligned");
+  cudaError_t e = ra::launch_int4_attention(P, in->q4, in->k4, in->v4t, in->sq, in->sk, in->sv, nullptr, ws, bh,
+                                            q_tile, kv_tile, s_out, p_out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "debug launch");
+}
+
+void ra_debug_set_wait_limit(uint32_t iterations) { g_wait_limit.store(iterations, std::memory_order_relaxed); }
+
+ra_status ra_debug_timeout_probe(void* ws, size_t ws_bytes, ra_stream stream) {
+  if (!aligned16(ws) || ws_bytes < sizeof(ra::WsHeader))
+    return fail(RA_ERR_INVALID_ARG, "workspace NULL, misaligned or too small");
+  cudaError_t e = ra::launch_timeout_probe(ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "timeout probe launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// ra_internal.h -- derived problem sizes, workspace layout and the launch
+// functions shared by the C ABI (ra_api.cu) and the kernel files.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ra_sm100.cuh"
+#include "../../include/rotate_attn.h"
+
+namespace ra {
+
+constexpr int D = 128;          // head_dim
+constexpr int QK_BLOCK = 64;    // tokens per Q/K quantisation block
+constexpr int TILE = 128;       // query rows per CTA tile and keys per KV tile
+
+// Problem with the sizes the kernels need, computed once on the host.
+struct Prob {
+  int B, H, BH;
+  int N, N_pad, n_video;
+  int F, Hh, W;
+  int split[3], off[3];         // segment sizes and first channel of each segment
+  int npos[3];                  // positions per axis: F, Hh, W
+  int tab_off[3];               // first table entry of each segment
+  int n_tab;                    // table entries (each: cos, sin, alpha, beta)
+  int rot;
+  uint64_t signature;
+};
+
+// Workspace layout (all offsets 256-byte aligned).
+struct WsHeader {
+  DeviceErr err;                // error word + first reporting site
+  uint32_t reserved0[2];
+  unsigned long long signature; // problem signature written by ra_prepare
+};
+
+struct WsLayout {
+  size_t tables;                // float4 [n_tab]
+  size_t vamax;                 // uint32 [BH][128]: fp32 bits of per-channel amax of V
+  size_t base_bytes;            // end of the part every call needs
+  size_t qr, kr, vt;            // FP16 path: fp16 [BH][N_pad][128] x2, fp16 [BH][128][N_pad]
+  size_t total_fp16;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const Prob& p) {
+  WsLayout L;
+  size_t o = align256(sizeof(WsHeader));
+  L.tables = o;
+  o = align256(o + sizeof(float) * 4 * (size_t)p.n_tab);
+  L.vamax = o;
+  o = align256(o + sizeof(uint32_t) * (size_t)p.BH * D);
+  L.base_bytes = o;
+  size_t plane = (size_t)p.BH * p.N_pad * D * 2;
+  L.qr = o;
+  o = align256(o + plane);
+  L.kr = o;
+  o = align256(o + plane);
+  L.vt = o;
+  o = align256(o + plane);
+  L.total_fp16 = o;
+  return L;
+}
+
+// Launches (stream-ordered; return the launch status).
+cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, const __half* v, uint8_t* q4,
+                            uint8_t* k4, uint8_t* v4t, float* sq, float* sk, float* sv, int32_t* vsum,
+                            void* ws, cudaStream_t st);
+cudaError_t launch_fp16_prologue(const Prob& p, const __half* q, const __half* k, const __half* v, void* ws,
+                                 cudaStream_t st);
+cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                                  const float* sq, const float* sk, const float* sv, __half* o, void* ws,
+                                  int dbg_bh, int dbg_qtile, int dbg_kv, int32_t* dbg_s, int8_t* dbg_p,
+                                  cudaStream_t st);
+cudaError_t launch_fp16_attention(const Prob& p, __half* o, void* ws, cudaStream_t st);
+cudaError_t launch_timeout_probe(void* ws, cudaStream_t st);
+
+// Iteration limit of every bounded device-side wait.
+uint32_t wait_limit();
+
+}  // namespace ra

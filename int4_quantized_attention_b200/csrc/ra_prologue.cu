@@ -1,0 +1,344 @@
+// ra_prologue.cu -- the fused prologue of the INT4 path and the FP16 path's
+// position encoding.  HBM-bound elementwise work: coalesced 16-byte loads,
+// per-element fp32 arithmetic with explicit round-to-nearest intrinsics (no
+// FMA contraction, IEEE division) so that codes and scales are reproducible
+// bit for bit, warp-shuffle block amax, packed INT4 stores.
+//
+// RotateAttention (arXiv 2607.02584) review page: 3D RoPE splits head_dim
+// into frame/height/width segments (core claim; axiom ledger); the
+// RoPE-aware rotation is block-diagonal 2x2 orthogonal, Interleaved on
+// adjacent dims (merged into RoPE) or Half, pairing each dim with its
+// counterpart in the other half of its segment (Fig. 3 caption); the blocks
+// are the 2x2 Hadamard (free-parameter ledger); Q and K are quantised to
+// symmetric INT4 per 64-token block, V per channel.
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "ra_internal.h"
+
+namespace ra {
+namespace {
+
+constexpr float kRsqrt2 = 0.70710678118654752440f;   // fp32 rounding of 1/sqrt(2)
+
+struct TokenPos {
+  int p[3];
+};
+
+__device__ __forceinline__ TokenPos token_pos(const Prob& P, int n) {
+  TokenPos t;
+  if (n >= P.n_video) {
+    t.p[0] = t.p[1] = t.p[2] = 0;   // text tokens: position 0 on every axis (no RoPE)
+  } else {
+    t.p[0] = n / (P.Hh * P.W);
+    t.p[1] = (n / P.W) % P.Hh;
+    t.p[2] = n % P.W;
+  }
+  return t;
+}
+
+__device__ __forceinline__ int segment_of(const Prob& P, int c) {
+  return c < P.off[1] ? 0 : (c < P.off[2] ? 1 : 2);
+}
+
+__device__ __forceinline__ void h8_to_f(const uint4& u, float (&f)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Symmetric INT4 code: clamp(rne(v / s), -7, 7); 0 when s == 0.
+__device__ __forceinline__ int int4_code(float v, float s) {
+  if (s == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(v, s));
+  return q > 7 ? 7 : (q < -7 ? -7 : q);
+}
+
+__device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P, uint32_t site) {
+  if (hdr->signature == P.signature) return true;
+  if (threadIdx.x == 0) report(const_cast<DeviceErr*>(&hdr->err), DEVERR_WORKSPACE, site);
+  return false;
+}
+
+// RoPE of the 4 adjacent pairs held by one thread (channels c0..c0+7 of
+// token n); with MERGED the coefficient is the Interleaved H2*Rot form.
+template <bool MERGED>
+__device__ __forceinline__ void rope8(const Prob& P, const float4* __restrict__ tab, const TokenPos& tp, int c0,
+                                      const float (&x)[8], float (&y)[8]) {
+#pragma unroll
+  for (int pp = 0; pp < 4; ++pp) {
+    const int c = c0 + 2 * pp;
+    const int s = segment_of(P, c);
+    const int j = (c - P.off[s]) >> 1;
+    const float4 t = __ldg(&tab[P.tab_off[s] + tp.p[s] * (P.split[s] >> 1) + j]);
+    const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
+    if (MERGED) {   // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
+      y[2 * pp] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
+      y[2 * pp + 1] = __fsub_rn(__fmul_rn(t.w, x0), __fmul_rn(t.z, x1));
+    } else {        // y0 = c x0 - s x1, y1 = s x0 + c x1
+      y[2 * pp] = __fsub_rn(__fmul_rn(t.x, x0), __fmul_rn(t.y, x1));
+      y[2 * pp + 1] = __fadd_rn(__fmul_rn(t.y, x0), __fmul_rn(t.x, x1));
+    }
+  }
+}
+
+__device__ __forceinline__ float block_max_128(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+}
+
+// One CTA = one 64-token block of Q or K of one head (128 threads).  Thread
+// t holds channels 8*(t%16) .. +7 of rows (t/16) + 8i, i = 0..7.
+template <int ROT>
+__global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __restrict__ q,
+                                                       const __half* __restrict__ k, uint8_t* __restrict__ q4,
+                                                       uint8_t* __restrict__ k4, float* __restrict__ sq,
+                                                       float* __restrict__ sk, const float4* __restrict__ tab,
+                                                       const WsHeader* __restrict__ hdr) {
+  __shared__ float red[4];
+  __shared__ float ys[ROT == RA_ROT_HALF ? QK_BLOCK : 1][ROT == RA_ROT_HALF ? D + 4 : 1];
+  if (!signature_ok(hdr, P, 0x100)) return;
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
+  uint8_t* out = (which ? k4 : q4) + (size_t)bh * P.N_pad * (D / 2);
+  float* scale = (which ? sk : sq) + (size_t)bh * (P.N_pad / QK_BLOCK);
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const int c0 = 8 * g;
+
+  uint4 raw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    raw[i] = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
+  }
+  float z[8][8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    float xf[8];
+    h8_to_f(raw[i], xf);
+    const TokenPos tp = token_pos(P, n < P.N ? n : 0);
+    rope8<ROT == RA_ROT_INTERLEAVED>(P, tab, tp, c0, xf, z[i]);
+  }
+  if (ROT == RA_ROT_HALF) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ys[r0 + 8 * i][c0 + e] = z[i][e];
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = c0 + e;
+      const int s = segment_of(P, c);
+      const int h = P.split[s] >> 1;
+      const bool first = (c - P.off[s]) < h;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = r0 + 8 * i;
+        const float a = first ? ys[r][c] : ys[r][c - h];
+        const float b = first ? ys[r][c + h] : ys[r][c];
+        z[i][e] = first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(z[i][e]));
+  amax = block_max_128(amax, red);
+  const float s = __fdiv_rn(amax, 7.0f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) packed |= (uint32_t)(int4_code(z[i][e], s) & 0xF) << (4 * e);
+    *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = packed;
+  }
+  if (threadIdx.x == 0) scale[blk] = s;
+}
+
+// Per-(head, channel) amax of V over a 256-token chunk, merged with
+// atomicMax on the bit pattern (valid for non-negative floats).
+__global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __restrict__ v,
+                                                     uint32_t* __restrict__ vamax,
+                                                     const WsHeader* __restrict__ hdr) {
+  __shared__ float part[8][D];
+  if (!signature_ok(hdr, P, 0x200)) return;
+  const int chunk = blockIdx.x, bh = blockIdx.y;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const __half* x = v + (size_t)bh * P.N * D;
+  float m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int i = 0; i < 32; ++i) {
+    const int n = chunk * 256 + r0 + 8 * i;
+    if (n >= P.N) break;
+    float f[8];
+    h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[r0][8 * g + e] = m[e];
+  __syncthreads();
+  const int c = threadIdx.x;
+  float r = part[0][c];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) r = fmaxf(r, part[i][c]);
+  atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
+}
+
+// One CTA = one 64-token block of V of one head: codes with the per-channel
+// scale, transposed packing (channel-major, two tokens per byte) and the
+// block's column sums.
+__global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
+                                                      const uint32_t* __restrict__ vamax,
+                                                      uint8_t* __restrict__ v4t, float* __restrict__ sv,
+                                                      int32_t* __restrict__ vsum,
+                                                      const WsHeader* __restrict__ hdr) {
+  __shared__ int8_t codes[QK_BLOCK][D + 16];
+  if (!signature_ok(hdr, P, 0x300)) return;
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const __half* x = v + (size_t)bh * P.N * D;
+  float s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    float f[8];
+    if (n < P.N) {
+      h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) codes[r0 + 8 * i][8 * g + e] = (int8_t)int4_code(f[e], s[e]);
+  }
+  __syncthreads();
+  const int c = threadIdx.x;
+  uint32_t w[8];
+  int sum = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int code = codes[8 * t + e][c];
+      sum += code;
+      word |= (uint32_t)(code & 0xF) << (4 * e);
+    }
+    w[t] = word;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(v4t + ((size_t)bh * D + c) * (P.N_pad / 2) + (size_t)blk * (QK_BLOCK / 2));
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
+  if (blk == 0) sv[(size_t)bh * D + c] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
+}
+
+// FP16 path: RoPE of Q and K rounded to fp16 ([BH][N_pad][128], padded rows
+// zero) and V transposed to [BH][128][N_pad] fp16 (padded tokens zero).
+__global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half* __restrict__ q,
+                                                            const __half* __restrict__ k,
+                                                            const __half* __restrict__ v, __half* __restrict__ qr,
+                                                            __half* __restrict__ kr, __half* __restrict__ vt,
+                                                            const float4* __restrict__ tab,
+                                                            const WsHeader* __restrict__ hdr) {
+  __shared__ __half tr[QK_BLOCK][D + 8];
+  if (!signature_ok(hdr, P, 0x400)) return;
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const int c0 = 8 * g;
+  const __half* x = (which == 0 ? q : which == 1 ? k : v) + (size_t)bh * P.N * D;
+  if (which < 2) {
+    __half* out = (which == 0 ? qr : kr) + (size_t)bh * P.N_pad * D;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int n = blk * QK_BLOCK + r0 + 8 * i;
+      uint4 o = make_uint4(0, 0, 0, 0);
+      if (n < P.N) {
+        float xf[8], y[8];
+        h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)), xf);
+        rope8<false>(P, tab, token_pos(P, n), c0, xf, y);
+        __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
+      }
+      *reinterpret_cast<uint4*>(out + (size_t)n * D + c0) = o;
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + 8 * i, n = blk * QK_BLOCK + r;
+    uint4 u = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
+    const __half* h = reinterpret_cast<const __half*>(&u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tr[r][c0 + e] = h[e];
+  }
+  __syncthreads();
+  // thread c writes channel c's 64 tokens (128 bytes) of this block
+  const int c = threadIdx.x;
+  __half* dst = vt + ((size_t)bh * D + c) * P.N_pad + (size_t)blk * QK_BLOCK;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    uint4 o;
+    __half* h = reinterpret_cast<__half*>(&o);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) h[e] = tr[8 * t + e][c];
+    reinterpret_cast<uint4*>(dst)[t] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, const __half* v, uint8_t* q4,
+                            uint8_t* k4, uint8_t* v4t, float* sq, float* sk, float* sv, int32_t* vsum, void* ws,
+                            cudaStream_t st) {
+  const WsLayout L = ws_layout(p);
+  char* base = static_cast<char*>(ws);
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(base);
+  const float4* tab = reinterpret_cast<const float4*>(base + L.tables);
+  uint32_t* vamax = reinterpret_cast<uint32_t*>(base + L.vamax);
+  const dim3 gqk(p.N_pad / QK_BLOCK, p.BH, 2);
+  switch (p.rot) {
+    case RA_ROT_NONE: qk_quant_kernel<RA_ROT_NONE><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    case RA_ROT_INTERLEAVED:
+      qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      break;
+    default: qk_quant_kernel<RA_ROT_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, st);
+  if (e != cudaSuccess) return e;
+  v_amax_kernel<<<dim3((p.N + 255) / 256, p.BH), 128, 0, st>>>(p, v, vamax, hdr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  v_quant_kernel<<<dim3(p.N_pad / QK_BLOCK, p.BH), 128, 0, st>>>(p, v, vamax, v4t, sv, vsum, hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp16_prologue(const Prob& p, const __half* q, const __half* k, const __half* v, void* ws,
+                                 cudaStream_t st) {
+  const WsLayout L = ws_layout(p);
+  char* base = static_cast<char*>(ws);
+  fp16_prologue_kernel<<<dim3(p.N_pad / QK_BLOCK, p.BH, 3), 128, 0, st>>>(
+      p, q, k, v, reinterpret_cast<__half*>(base + L.qr), reinterpret_cast<__half*>(base + L.kr),
+      reinterpret_cast<__half*>(base + L.vt), reinterpret_cast<const float4*>(base + L.tables),
+      reinterpret_cast<const WsHeader*>(base));
+  return cudaGetLastError();
+}
+
+}  // namespace ra

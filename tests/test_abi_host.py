@@ -1,0 +1,120 @@
+"""Host-only checks of the C ABI: the library builds and loads, exports every
+function the header declares, validates arguments before touching the GPU,
+and builds RoPE/rotation tables identical to the oracle's."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from int4_quantized_attention_b200 import api, build, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "rotate_attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ra_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(lib):
+    names = header_functions()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in the header but not exported"
+    assert set(names) == set(api._SIGNATURES), "binding and header disagree"
+
+
+def test_library_is_sm100a(lib):
+    # the build flags target sm_100a only
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.NVCC_FLAGS)
+
+
+def prob(**kw):
+    return api.problem(synth.CONFIGS["tiny"].replace(**kw))
+
+
+def test_validation_codes(lib):
+    assert api.validate(prob()) == api.RA_OK
+    assert api.validate(prob(d=64)) == api.RA_ERR_UNSUPPORTED
+    assert api.validate(prob(split=(44, 42, 40))) == api.RA_ERR_INVALID_ARG   # sum != d
+    assert api.validate(prob(split=(43, 43, 42))) == api.RA_ERR_INVALID_ARG   # odd
+    assert api.validate(prob(F=0, Hh=0, W=0, n_text=0)) == api.RA_ERR_INVALID_ARG   # N = 0
+    assert api.validate(prob(H=0)) == api.RA_ERR_INVALID_ARG
+    assert api.validate(prob(theta=0.0)) == api.RA_ERR_INVALID_ARG
+    p = prob()
+    p.rot = 7
+    assert api.validate(p) == api.RA_ERR_INVALID_ARG
+    assert api.validate(prob(F=0, Hh=0, W=0, n_text=5)) == api.RA_OK          # text only
+    assert api.validate(prob(F=2, Hh=0, W=3, n_text=5)) == api.RA_ERR_INVALID_ARG
+    api.validate(prob(split=(44, 42, 40)))
+    assert b"split" in lib.ra_last_error_detail()
+
+
+def test_sizes(lib):
+    for name, cfg in synth.CONFIGS.items():
+        p = api.problem(cfg)
+        assert api.seq_len(p) == cfg.N
+        assert api.seq_pad(p) == (cfg.N + 127) // 128 * 128
+        Np, BH = api.seq_pad(p), cfg.B * cfg.H
+        min_qkv = 3 * BH * Np * 64 + 2 * BH * (Np // 64) * 4 + BH * 128 * 4 + BH * (Np // 64) * 128 * 4
+        assert api.qkv4_bytes(p) >= min_qkv
+        assert api.workspace_bytes(p, True) >= api.workspace_bytes(p, False) + 3 * BH * Np * 128 * 2
+
+
+def test_calls_reject_bad_arguments_without_a_gpu(lib):
+    p = prob()
+    q = api.Qkv4()
+    ws = ctypes.c_void_p(None)
+    st = lib.ra_rotate_quantize_qkv(ctypes.byref(p), None, None, None, ctypes.byref(q), ws, 0, None)
+    assert st == api.RA_ERR_INVALID_ARG
+    st = lib.ra_int4_attention_fwd(ctypes.byref(p), ctypes.byref(q), None, ws, 0, None)
+    assert st == api.RA_ERR_INVALID_ARG
+    st = lib.ra_fp16_attention_fwd(ctypes.byref(p), 16, 16, 16, 16, 32, 10, None)
+    assert st == api.RA_ERR_WORKSPACE                 # undersized workspace
+    st = lib.ra_fp16_attention_fwd(ctypes.byref(p), 17, 16, 16, 16, 32, 1 << 40, None)
+    assert st == api.RA_ERR_INVALID_ARG               # misaligned q
+    st = lib.ra_prepare(ctypes.byref(p), 32, 16, None)
+    assert st == api.RA_ERR_WORKSPACE
+    bad = prob(d=96)
+    st = lib.ra_int4_attention_fwd(ctypes.byref(bad), ctypes.byref(q), 16, 32, 1 << 40, None)
+    assert st == api.RA_ERR_UNSUPPORTED
+    buf = api.Qkv4()
+    st = lib.ra_qkv4_bind(ctypes.byref(p), 256, 10, ctypes.byref(buf))
+    assert st == api.RA_ERR_INVALID_ARG
+    st = lib.ra_qkv4_bind(ctypes.byref(p), 512, 1 << 30, ctypes.byref(buf))
+    assert st == api.RA_OK and buf.q4 == 512 and buf.k4 > buf.q4
+    st = lib.ra_debug_int4_tile(ctypes.byref(p), ctypes.byref(buf), 0, 5, 0, 16, 16, 32, 1 << 40, None)
+    assert st == api.RA_ERR_INVALID_ARG               # q tile out of range (N_pad/128 = 2)
+    for s in range(7):
+        assert api.status_string(s)
+
+
+@pytest.mark.parametrize("name", ["tiny", "half", "wan", "hunyuan"])
+def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
+    cfg = synth.CONFIGS[name]
+    tab = api.build_tables_host(api.problem(cfg))
+    npos = (cfg.F, cfg.Hh, cfg.W)
+    k = 0
+    rng = np.random.default_rng(0)
+    for s in range(3):
+        half = cfg.split[s] // 2
+        # every entry for small grids, a sample for the large ones
+        cells = [(pos, j) for pos in range(npos[s]) for j in range(half)]
+        if len(cells) > 400:
+            idx = rng.choice(len(cells), 400, replace=False)
+            cells = [cells[i] for i in idx] + [(npos[s] - 1, half - 1)]
+        for pos, j in cells:
+            ref = np.array(oracle_mod.rope_coef(cfg, s, pos, j), np.float32)
+            got = tab[k + pos * half + j]
+            assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (name, s, pos, j)
+        k += npos[s] * half
+    assert k == len(tab)

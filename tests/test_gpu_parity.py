@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars:
+  * prologue (INT4 codes, block scales, V channel scales, V column sums):
+    bit-exact on every element;
+  * int32 S = Q K^T tiles: bit-exact (through the debug export);
+  * P codes: equal except rare +-1 flips where 15 P sits within float
+    rounding of a .5 boundary (the kernel's exp2 is the hardware's);
+  * fp16 output: cosine >= 0.9999 and max |err| <= 2e-2 * max|V| against the
+    oracle; the FP16 path: cosine >= 0.9999, max |err| <= 1e-2 * max|V|.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from int4_quantized_attention_b200 import api, build, synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+COS_MIN = 0.9999
+MAXABS_INT4 = 2e-2
+MAXABS_FP16 = 1e-2
+P_FLIP_MAX = 1e-3      # fraction of valid P codes allowed to differ (each by +-1)
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    api.lib()
+    return torch.device("cuda:0")
+
+
+def cosine(a, b):
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
+
+
+def to_dev(x, dev):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+
+def run_int4(cfg, dev, q, k, v):
+    ra = api.RotateAttention(cfg, dev, fp16_path=False)
+    qd, kd, vd = (to_dev(t, dev) for t in (q, k, v))
+    ra.rotate_quantize(qd, kd, vd)
+    o = ra.int4_attention()
+    ra.check()
+    return ra, o.cpu().numpy()
+
+
+def oracle_head(oracle_mod, cfg, q, k, v, b, h):
+    return oracle_mod.quantize_head(cfg, q[b, h], k[b, h], v[b, h])
+
+
+def check_prologue(oracle_mod, cfg, got, q, k, v, heads):
+    N, Np = cfg.N, (cfg.N + 127) // 128 * 128
+    for bh in heads:
+        b, h = divmod(bh, cfg.H)
+        ref = oracle_head(oracle_mod, cfg, q, k, v, b, h)
+        for key in ("qc", "kc", "vc"):
+            assert np.array_equal(got[key][bh], ref[key]), (key, bh, np.argwhere(got[key][bh] != ref[key])[:5])
+        for key in ("qs", "ks", "sv"):
+            assert np.array_equal(got[key][bh].view(np.uint32), ref[key].view(np.uint32)), (key, bh)
+        assert np.array_equal(got["colsum"][bh], ref["colsum"]), ("colsum", bh)
+        yield bh, ref
+
+
+SMALL = {
+    "tiny": synth.CONFIGS["tiny"],
+    "half": synth.CONFIGS["half"],
+    # ragged: N = 3*7*9 + 5 = 194 (N mod 64 = 2), interleaved
+    "ragged_text": synth.Config("ragged_text", 1, 3, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 11),
+    # HunyuanVideo split with text tokens, half rotation, N = 2*9*10 + 40 = 220
+    "hy_split": synth.Config("hy_split", 1, 2, 2, 9, 10, 40, (16, 56, 56), "half", "lognormal1.5", 12),
+    # no rotation, batch 2, a single partial tile (N = 90)
+    "norot_b2": synth.Config("norot_b2", 2, 2, 2, 5, 9, 0, (44, 42, 42), "none", "lognormal1", 13),
+    # text-only sequence (no video grid), N = 130: two tiles, second has 2 keys
+    "text_only": synth.Config("text_only", 1, 1, 0, 0, 0, 130, (44, 42, 42), "half", "outlier8", 14),
+    # several tiles: N = 4*16*20 = 1280
+    "multi_tile": synth.Config("multi_tile", 1, 2, 4, 16, 20, 0, (44, 42, 42), "interleaved", "lognormal1.5", 15),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_int4_path_matches_oracle(oracle_mod, dev, name):
+    cfg = SMALL[name]
+    q, k, v = synth.make_qkv(cfg)
+    ra, o = run_int4(cfg, dev, q, k, v)
+    got = ra.unpack()
+    BH, N = cfg.B * cfg.H, cfg.N
+    worst_cos, worst_err = 1.0, 0.0
+    for bh, ref in check_prologue(oracle_mod, cfg, got, q, k, v, range(BH)):
+        b, h = divmod(bh, cfg.H)
+        out_ref, out64 = oracle_mod.attention_rows(cfg, ref, want64=True)
+        g = o[b, h].astype(np.float64)
+        c = cosine(g, out64)
+        err = np.abs(g - out64).max() / np.abs(v[b, h].astype(np.float64)).max()
+        worst_cos, worst_err = min(worst_cos, c), max(worst_err, err)
+    assert worst_cos >= COS_MIN, worst_cos
+    assert worst_err <= MAXABS_INT4, worst_err
+
+
+@pytest.mark.parametrize("name", ["tiny", "half", "ragged_text", "text_only", "multi_tile"])
+def test_int4_S_tiles_bit_exact_and_P_codes(oracle_mod, dev, name):
+    cfg = SMALL[name]
+    q, k, v = synth.make_qkv(cfg)
+    ra, _ = run_int4(cfg, dev, q, k, v)
+    BH, Np = cfg.B * cfg.H, (cfg.N + 127) // 128 * 128
+    nt = Np // 128
+    flips = total = 0
+    cases = {(0, 0, 0), (0, nt - 1, nt - 1), (BH - 1, 0, nt - 1), (BH - 1, nt - 1, 0)}
+    refs = {}
+    for bh, qt, kt in sorted(cases):
+        S, P = api.debug_int4_tile(ra.p, ra.qkv4, bh, qt, kt, ra.workspace)
+        ra.check()
+        S, P = S.cpu().numpy(), P.cpu().numpy()
+        b, h = divmod(bh, cfg.H)
+        if bh not in refs:
+            refs[bh] = oracle_head(oracle_mod, cfg, q, k, v, b, h)
+        for r in range(128):
+            i = qt * 128 + r
+            if i >= cfg.N:
+                continue
+            Sr, Pr = oracle_mod.attention_row_debug(cfg, refs[bh], i, kt)
+            assert np.array_equal(S[r], Sr), (bh, qt, kt, r)
+            valid = Pr != -128
+            assert np.array_equal(P[r][~valid], Pr[~valid])
+            d = np.abs(P[r][valid].astype(int) - Pr[valid].astype(int))
+            assert d.max(initial=0) <= 1
+            flips += int((d > 0).sum())
+            total += int(valid.sum())
+    assert flips <= P_FLIP_MAX * total + 2, (flips, total)
+
+
+@pytest.mark.parametrize("name", ["tiny", "hy_split", "multi_tile", "text_only"])
+def test_fp16_path_matches_oracle(oracle_mod, dev, name):
+    cfg = SMALL[name]
+    q, k, v = synth.make_qkv(cfg)
+    ra = api.RotateAttention(cfg, dev, fp16_path=True)
+    o = ra.fp16_attention(*(to_dev(t, dev) for t in (q, k, v)))
+    ra.check()
+    o = o.cpu().numpy()
+    for bh in range(cfg.B * cfg.H):
+        b, h = divmod(bh, cfg.H)
+        ref = oracle_mod.fp16_attention_rows(cfg, q[b, h], k[b, h], v[b, h])
+        g = o[b, h].astype(np.float64)
+        assert cosine(g, ref) >= COS_MIN
+        assert np.abs(g - ref).max() <= MAXABS_FP16 * np.abs(v[b, h].astype(np.float64)).max()
+
+
+def test_int4_path_is_deterministic(dev):
+    cfg = SMALL["multi_tile"]
+    q, k, v = synth.make_qkv(cfg)
+    _, o1 = run_int4(cfg, dev, q, k, v)
+    _, o2 = run_int4(cfg, dev, q, k, v)
+    assert np.array_equal(o1.view(np.uint16), o2.view(np.uint16))
+
+
+def test_device_timeout_is_reported_not_hung(dev):
+    cfg = SMALL["tiny"]
+    ra = api.RotateAttention(cfg, dev, fp16_path=False)
+    api.debug_set_wait_limit(1)
+    try:
+        api.debug_timeout_probe(ra.workspace)
+        with pytest.raises(api.RotateAttnError) as e:
+            ra.check()
+        assert e.value.status == api.RA_ERR_DEVICE_TIMEOUT
+    finally:
+        api.debug_set_wait_limit(0)
+    ra.check()          # cleared; the context is still usable
+    q, k, v = synth.make_qkv(cfg)
+    run_int4(cfg, dev, q, k, v)
+
+
+def test_unprepared_workspace_is_reported(dev):
+    cfg = SMALL["tiny"]
+    ra = api.RotateAttention(cfg, dev, fp16_path=False)
+    other = api.problem(cfg.replace(theta=500.0))      # same sizes, different RoPE base
+    q, k, v = (to_dev(t, dev) for t in synth.make_qkv(cfg))
+    api.rotate_quantize_qkv(other, q, k, v, ra.qkv4, ra.workspace)
+    with pytest.raises(api.RotateAttnError) as e:
+        ra.check()
+    assert e.value.status == api.RA_ERR_WORKSPACE
+
+
+# ------------------------------------------------------------------ full size
+
+FULL = ["wan", "hunyuan"]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(oracle_mod, dev, name):
+    """Full-size workload in the benchmark's launch configuration: every
+    prologue element bit-exact; output rows sampled (head 0 and the last head
+    densely, a few rows of every other head, always the ragged last row)."""
+    cfg = synth.CONFIGS[name]
+    q, k, v = synth.make_qkv(cfg)
+    ra, o = run_int4(cfg, dev, q, k, v)
+    got = ra.unpack()
+    BH, N = cfg.B * cfg.H, cfg.N
+    rng = np.random.default_rng(99)
+    heads = list(range(BH))
+    for bh, ref in check_prologue(oracle_mod, cfg, got, q, k, v, heads):
+        b, h = divmod(bh, cfg.H)
+        nrows = 96 if bh in (0, BH - 1) else 4
+        rows = np.unique(np.concatenate([rng.choice(N, nrows, replace=False), [0, N - 1]])).astype(np.int64)
+        _, out64 = oracle_mod.attention_rows(cfg, ref, rows=rows, want64=True)
+        g = o[b, h][rows].astype(np.float64)
+        assert cosine(g, out64) >= COS_MIN, (bh, cosine(g, out64))
+        assert np.abs(g - out64).max() <= MAXABS_INT4 * np.abs(v[b, h].astype(np.float64)).max()
