@@ -99,7 +99,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_oracle_sample(cfg, budget_s: float = 12.0, max_rows: int = 4096):
+def cpu_oracle_sample(cfg, budget_s: float = 12.0, max_rows: int = 65536):
     """Time the oracle on a bounded sample: the prologue of head 0 and the
     INT4 attention of query rows of head 0, in batches until the budget."""
     from oracle import oracle as O
