@@ -141,6 +141,36 @@ ra_status ra_check_device_error(void *workspace, ra_stream stream);
 const char *ra_status_string(ra_status s);
 const char *ra_last_error_detail(void);
 
+/* ---- allocation-free prologue ------------------------------------------ */
+
+/* Size of the fixed device scratch behind ra_rotate_quantize_qkv_noalloc. */
+#define RA_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/* The same fused prologue as ra_rotate_quantize_qkv (same kernels, same
+ * bit-exact outputs), for callers that cannot give the library any device
+ * memory beyond their own inputs and outputs: for example an engine plugin
+ * whose enqueue hook must not allocate (cudaMalloc may synchronise the device
+ * or fail mid-run), or a program whose device memory is fully laid out in
+ * advance.  The paper has no counterpart; this is a deployment variant.
+ *
+ * Its scratch -- error word, RoPE/rotation tables and the per-channel V amax
+ * -- lives in one fixed array of RA_NOALLOC_SCRATCH_BYTES inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Problems whose scratch would not fit (about 512 bytes per head plus
+ * 16 bytes per RoPE table entry, plus a 256-byte header) are rejected with
+ * RA_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine); it copies the
+ * tables from static host memory with cudaMemcpyAsync on `stream`, then
+ * launches the prologue.  The first call on each device also looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture.  Every call shares the one
+ * array and leaves its contents behind; what must start at zero (the error
+ * word, the V amax) is cleared by each call.  Calls whose GPU work overlaps
+ * (other streams, other host threads) race on the array: serialise them.
+ * q, k, v, out: as for ra_rotate_quantize_qkv. */
+ra_status ra_rotate_quantize_qkv_noalloc(const ra_problem *p, const void *q, const void *k, const void *v,
+                                         const ra_qkv4 *out, ra_stream stream);
+
 /* ---- test hooks ------------------------------------------------------- */
 
 /* Number of floats of the coefficient table and the table itself, as

@@ -63,6 +63,7 @@ _SIGNATURES = {
     "ra_build_tables_host": (ctypes.c_int, [_P, _V, _SZ]),
     "ra_debug_int4_tile": (ctypes.c_int, [_P, ctypes.POINTER(Qkv4), ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _V, _V, _V, _SZ, _V]),
+    "ra_rotate_quantize_qkv_noalloc": (ctypes.c_int, [_P, _V, _V, _V, ctypes.POINTER(Qkv4), _V]),
     "ra_debug_set_wait_limit": (None, [ctypes.c_uint32]),
     "ra_debug_timeout_probe": (ctypes.c_int, [_V, _SZ, _V]),
 }
@@ -163,6 +164,13 @@ def fp16_attention_fwd(p: Problem, q, k, v, o, workspace, stream=None) -> None:
     _check("ra_fp16_attention_fwd",
            lib().ra_fp16_attention_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(workspace),
                                        workspace.numel(), _stream(stream)))
+
+
+def rotate_quantize_qkv_noalloc(p: Problem, q, k, v, out: Qkv4, stream=None) -> None:
+    """The prologue with its scratch in the library's fixed device array."""
+    _check("ra_rotate_quantize_qkv_noalloc",
+           lib().ra_rotate_quantize_qkv_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), ctypes.byref(out),
+                                                _stream(stream)))
 
 
 def check_device_error(workspace, stream=None) -> None:

@@ -168,6 +168,9 @@ uint32_t wait_limit() {
   const uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
   return v ? v : kDefaultWaitLimit;
 }
+ra_status derive_problem(const ra_problem* p, Prob* out) { return derive(p, out); }
+void build_coef_tables(const ra_problem* p, const Prob& P, float* out) { build_tables(p, P, out); }
+void set_error_detail(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
 }  // namespace ra
 
 extern "C" {

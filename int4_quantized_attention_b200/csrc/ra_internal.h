@@ -79,4 +79,10 @@ cudaError_t launch_timeout_probe(void* ws, cudaStream_t st);
 // Iteration limit of every bounded device-side wait.
 uint32_t wait_limit();
 
+// Host helpers shared with the allocation-free entry point (ra_noalloc.cu):
+// problem validation with derived sizes, and the coefficient table builder.
+ra_status derive_problem(const ra_problem* p, Prob* out);
+void build_coef_tables(const ra_problem* p, const Prob& P, float* out);
+void set_error_detail(const char* msg);
+
 }  // namespace ra
