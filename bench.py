@@ -188,6 +188,11 @@ def our_arm(args, cfg, rank, world):
         ms_pro = event_time(lambda: ra.rotate_quantize(qd, kd, vd), max(args.steps, 10), stream)
     ra.check()
     torch.cuda.synchronize()
+    if args.only_step:
+        if rank == 0:
+            print(json.dumps({"workload": cfg.name, "ms_per_step": ms_step, "int4_attention_ms": ms_attn,
+                              "prologue_ms": ms_pro}), flush=True)
+        return
     if world > 1:
         t = torch.tensor([ms_step], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -303,9 +308,14 @@ def main():
     ap.add_argument("--config", default="wan", choices=sorted(synth.CONFIGS))
     ap.add_argument("--schedule", action="store_true", help="also run the 400-call mixed schedule")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
+    ap.add_argument("--only-step", action="store_true",
+                    help="run only the warm-up and timed INT4 steps (for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = synth.CONFIGS[args.config]
+    if args.heads:
+        cfg = cfg.replace(H=args.heads, name=f"{cfg.name}-H{args.heads}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

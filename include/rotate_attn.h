@@ -67,8 +67,10 @@ typedef struct {
  *   q4, k4 : uint8 [B][H][N_pad][64]  two INT4 codes per byte, channel 2c in
  *            the low nibble and 2c+1 in the high nibble, two's complement,
  *            codes in [-7, 7]
- *   v4t    : uint8 [B][H][128][N_pad/2]  V transposed (channel-major), token
- *            2t in the low nibble and 2t+1 in the high nibble
+ *   v4t    : uint8 [B][H][N_pad/128][128][64]  V transposed per 128-token
+ *            tile: tile t, channel c, byte b holds tokens 128t+2b (low
+ *            nibble) and 128t+2b+1 (high nibble); each tile is one contiguous
+ *            8 KB block
  *   sq, sk : float [B][H][N_pad/64]   one scale per 64-token block (amax/7)
  *   sv     : float [B][H][128]        one scale per channel over all N tokens
  *   vsum   : int32 [B][H][N_pad/64][128]  per-64-token-block column sums of
@@ -188,11 +190,11 @@ ra_status ra_debug_int4_tile(const ra_problem *p, const ra_qkv4 *in, int bh, int
                              int32_t *s_out, int8_t *p_out, void *workspace, size_t workspace_bytes,
                              ra_stream stream);
 
-/* Sets the iteration limit of every bounded device-side wait (0 restores the
- * default); a test sets 1 and runs ra_debug_timeout_probe, whose kernel waits
- * on a barrier that nothing arms and must return RA_ERR_DEVICE_TIMEOUT via
- * ra_check_device_error. */
-void ra_debug_set_wait_limit(uint32_t iterations);
+/* Sets the wall-clock limit of every bounded device-side wait, in
+ * microseconds (0 restores the default of 2 s); a test sets 1 and runs
+ * ra_debug_timeout_probe, whose kernel waits on a barrier that nothing arms
+ * and must return RA_ERR_DEVICE_TIMEOUT via ra_check_device_error. */
+void ra_debug_set_wait_timeout_us(uint32_t microseconds);
 ra_status ra_debug_timeout_probe(void *workspace, size_t workspace_bytes, ra_stream stream);
 
 #ifdef __cplusplus

@@ -64,7 +64,7 @@ _SIGNATURES = {
     "ra_debug_int4_tile": (ctypes.c_int, [_P, ctypes.POINTER(Qkv4), ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _V, _V, _V, _SZ, _V]),
     "ra_rotate_quantize_qkv_noalloc": (ctypes.c_int, [_P, _V, _V, _V, ctypes.POINTER(Qkv4), _V]),
-    "ra_debug_set_wait_limit": (None, [ctypes.c_uint32]),
+    "ra_debug_set_wait_timeout_us": (None, [ctypes.c_uint32]),
     "ra_debug_timeout_probe": (ctypes.c_int, [_V, _SZ, _V]),
 }
 
@@ -198,8 +198,8 @@ def debug_int4_tile(p: Problem, qkv4: Qkv4, bh: int, q_tile: int, kv_tile: int, 
     return s_out, p_out
 
 
-def debug_set_wait_limit(iterations: int) -> None:
-    lib().ra_debug_set_wait_limit(iterations)
+def debug_set_wait_timeout_us(microseconds: int) -> None:
+    lib().ra_debug_set_wait_timeout_us(microseconds)
 
 
 def debug_timeout_probe(workspace, stream=None) -> None:
@@ -271,13 +271,13 @@ class RotateAttention:
         packed = BH * Np * 64
         q4 = view(self.qkv4.q4, packed, np.uint8).reshape(BH, Np, 64)
         k4 = view(self.qkv4.k4, packed, np.uint8).reshape(BH, Np, 64)
-        v4t = view(self.qkv4.v4t, packed, np.uint8).reshape(BH, 128, Np // 2)
+        v4t = view(self.qkv4.v4t, packed, np.uint8).reshape(BH, Np // 128, 128, 64)
         sq = view(self.qkv4.sq, BH * (Np // 64) * 4, np.float32).reshape(BH, Np // 64)
         sk = view(self.qkv4.sk, BH * (Np // 64) * 4, np.float32).reshape(BH, Np // 64)
         sv = view(self.qkv4.sv, BH * 128 * 4, np.float32).reshape(BH, 128)
         vsum = view(self.qkv4.vsum, BH * (Np // 64) * 128 * 4, np.int32).reshape(BH, Np // 64, 128)
         return dict(qc=unpack_nibbles(q4), kc=unpack_nibbles(k4),
-                    vc=np.ascontiguousarray(unpack_nibbles(v4t).transpose(0, 2, 1)),
+                    vc=np.ascontiguousarray(unpack_nibbles(v4t).transpose(0, 1, 3, 2).reshape(BH, Np, 128)),
                     qs=sq, ks=sk, sv=sv, colsum=vsum)
 
 

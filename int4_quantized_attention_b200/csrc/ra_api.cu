@@ -16,8 +16,8 @@
 namespace {
 
 thread_local char g_detail[256] = "";
-std::atomic<uint32_t> g_wait_limit{0};
-constexpr uint32_t kDefaultWaitLimit = 1u << 22;   // polls of mbarrier.try_wait (about a second)
+std::atomic<uint32_t> g_wait_limit_us{0};
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // 2 s of wall-clock time per wait
 
 ra_status fail(ra_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 ra_status fail(ra_status s, const char* fmt, ...) {
@@ -164,9 +164,9 @@ ra_status check_qkv4(const ra_qkv4* t) {
 }  // namespace
 
 namespace ra {
-uint32_t wait_limit() {
-  const uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
-  return v ? v : kDefaultWaitLimit;
+uint64_t wait_limit() {
+  const uint32_t us = g_wait_limit_us.load(std::memory_order_relaxed);
+  return us ? 1000ull * us : kDefaultWaitLimitNs;
 }
 ra_status derive_problem(const ra_problem* p, Prob* out) { return derive(p, out); }
 void build_coef_tables(const ra_problem* p, const Prob& P, float* out) { build_tables(p, P, out); }
@@ -351,7 +351,9 @@ ra_status ra_debug_int4_tile(const ra_problem* p, const ra_qkv4* in, int bh, int
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "debug launch");
 }
 
-void ra_debug_set_wait_limit(uint32_t iterations) { g_wait_limit.store(iterations, std::memory_order_relaxed); }
+void ra_debug_set_wait_timeout_us(uint32_t microseconds) {
+  g_wait_limit_us.store(microseconds, std::memory_order_relaxed);
+}
 
 ra_status ra_debug_timeout_probe(void* ws, size_t ws_bytes, ra_stream stream) {
   if (!aligned16(ws) || ws_bytes < sizeof(ra::WsHeader))

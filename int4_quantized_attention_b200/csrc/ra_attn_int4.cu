@@ -1,0 +1,523 @@
+// ra_attn_int4.cu -- INT4 attention forward, warp-specialised, on the sm_100a
+// 5th-generation tensor cores.
+//
+// RotateAttention (arXiv 2607.02584) review page: INT4 FlashAttention with
+// online softmax (abstract); range-optimised P quantisation -- P = exp(s - m)
+// in [0, 1] mapped to rne(15 P) - 8 in [-8, 7], fixed scale 15, zero-point -8
+// (Sec. 4.2 as summarised by the referee report; free-parameter ledger) --
+// with the zero-point corrected through the V column sums.
+//
+// One CTA = one (batch*head, pair of 128-row query tiles A and B); 512
+// threads in four warpgroups:
+//   WG0 (warps 0-3)    softmax of tile A, thread t = query row t = TMEM lane t
+//   WG1 (warps 4-7)    softmax of tile B
+//   WG2 (warps 8-11)   widen packed INT4 K and V^T tiles into INT8 (16*code)
+//                      in 128-byte-swizzled K-major SMEM operands, 4 stages
+//   WG3 warp 12        bulk-copy producer (packed K, V^T tiles, 8 KB each,
+//                      into a 3-stage ring; the two packed Q tiles once)
+//       warp 13        TMEM owner and single-thread tcgen05.mma issuer
+// TMEM (512 columns): S_A | S_B | O_A | O_B, 128 int32 columns each.  The P
+// operand of a tile (128 rows x 128 u8 = 32 columns) is stored by the softmax
+// threads into the last 32 columns of their own S region once S is in
+// registers, and read from there by the P.V MMA (A operand in TMEM).
+// MMA order per query tile X: S_X(0); then for every tile j: O_X += W_X(j)
+// V(j), S_X(j+1) -- tiles A and B interleaved, so the tensor core runs one
+// tile's MMAs while the other tile's softmax runs (ping-pong).  Because the
+// MMAs of one CTA complete in issue order, the arrival of S_X(j+1) also means
+// that P.V(j) has landed: the softmax may rescale O_X right then.
+//
+// The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15], fed as an
+// unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
+// sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
+// The int32 P.V accumulator stays in TMEM across tiles; a row whose running
+// max moves rescales its accumulator in place with an integer multiply by
+// round(2^30 * exp(m_old - m_new)) (exp(...) is exactly 1 for every other
+// row).  The normaliser l is the running sum of w.
+//
+// INT4 codes are widened to 16*code (the nibble placed in the high half of
+// the byte), so S comes out as 256*S and P.V as 16*P.V, exactly; both factors
+// fold into the dequantisation.  Within every 8-element group the widened
+// operands hold even elements first, then odd ones (channels for Q and K,
+// keys for V^T); the P operand is packed in the same key order.
+//
+// Keys past N (the ragged last tile) hold zero K and V codes: their P.V
+// contribution is zero whatever their w, so only the max and the normaliser
+// must exclude them; their P bytes are zeroed as well.
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "ra_internal.h"
+
+namespace ra {
+namespace {
+
+constexpr int NUM_THREADS = 512;
+constexpr int PK_STAGES = 3;   // packed K/V^T staging (bulk copies)
+constexpr int OP_STAGES = 4;   // widened K/V^T operands
+// Register split: launched at LAUNCH_REGS per thread (512 x 128 = 65536); the
+// widen and producer warpgroups drop to PRODUCER_REGS, the two softmax
+// warpgroups rise to SOFTMAX_REGS: 256 x 200 + 256 x 56 = 65536.
+constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 200, PRODUCER_REGS = 56;
+static_assert(256 * SOFTMAX_REGS + 256 * PRODUCER_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
+
+constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
+constexpr uint32_t IDESC_PV = make_idesc(2, 0, 1, 128, 128);   // s32 += u8 x s8
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float SQRT_D = 11.313708498984761f;
+constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
+constexpr int MAGIC_BITS = 0x4B400000;
+constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6), still exact through MAGIC
+constexpr uint32_t P_COL = 96;    // P operand: columns 96..127 of the tile's S region
+
+struct Smem {
+  static constexpr uint32_t QA = 0, QB = 16384;   // widened Q tiles
+  static constexpr uint32_t OP = 32768;           // 4 x 32 KB: widened K (+0), V^T (+16 KB)
+  static constexpr uint32_t PK = 163840;          // 3 x 16 KB: packed K (+0), V^T (+8 KB)
+  static constexpr uint32_t QPK = 212992;         // 16 KB: packed Q staging
+  static constexpr uint32_t BAR = 229376;
+  static constexpr uint32_t BYTES = BAR + 256;
+};
+
+enum : int {
+  B_PK_FULL = 0, B_PK_EMPTY = 3, B_OP_FULL = 6, B_OP_EMPTY = 10, B_QPACK = 14, B_QFULL = 15,
+  B_S_FULL = 16, B_P_FULL = 18, B_O_DONE = 20, B_DRAIN = 22, NBAR = 23
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T for kind::i8: A holds 4 bytes of a row per
+// 32-bit column, row m in lane m.
+__device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 4 packed words (32 codes) -> two 16-byte chunks of 16*code, evens then odds
+// per 8-element group.
+__device__ __forceinline__ void widen16(const uint4 u, uint4& a, uint4& b) {
+  a = make_uint4((u.x << 4) & 0xF0F0F0F0u, u.x & 0xF0F0F0F0u, (u.y << 4) & 0xF0F0F0F0u, u.y & 0xF0F0F0F0u);
+  b = make_uint4((u.z << 4) & 0xF0F0F0F0u, u.z & 0xF0F0F0F0u, (u.w << 4) & 0xF0F0F0F0u, u.w & 0xF0F0F0F0u);
+}
+
+// P word k (0..31) holds, in byte b, key 8 (k / 2) + 2 b + (k % 2).  Byte mask
+// of the keys < nvalid.
+__device__ __forceinline__ uint32_t p_word_mask(int k, int nvalid) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int key = 8 * (k >> 1) + 2 * b + (k & 1);
+    m |= (key < nvalid ? 0xFFu : 0u) << (8 * b);
+  }
+  return m;
+}
+
+struct KernelArgs {
+  Prob P;
+  const uint8_t* q4;
+  const uint8_t* k4;
+  const uint8_t* v4t;
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  __half* o;
+  WsHeader* hdr;
+  uint64_t limit;
+  int dbg_bh, dbg_qt, dbg_kv;
+  int32_t* dbg_s;
+  int8_t* dbg_p;
+};
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Smem::BAR + 8 * NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::BAR + 8 * NBAR + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Prob& P = a.P;
+  const bool dbg_run = a.dbg_s != nullptr;
+  const int n_qt = P.N_pad / TILE, nt = n_qt, nblk = P.N_pad / QK_BLOCK;
+  const int qt0 = 2 * (blockIdx.x + (dbg_run ? a.dbg_qt / 2 : 0));
+  const int bh = blockIdx.y + (dbg_run ? a.dbg_bh : 0);
+  const bool hasB = qt0 + 1 < n_qt;
+  DeviceErr* err = &a.hdr->err;
+  const uint64_t limit = a.limit;
+
+  if (tid == 0) {
+    for (int i = 0; i < PK_STAGES; ++i) {
+      mbar_init(&bar[B_PK_FULL + i], 1);
+      mbar_init(&bar[B_PK_EMPTY + i], 4);
+    }
+    for (int i = 0; i < OP_STAGES; ++i) {
+      mbar_init(&bar[B_OP_FULL + i], 4);
+      mbar_init(&bar[B_OP_EMPTY + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[B_S_FULL + i], 1);
+      mbar_init(&bar[B_P_FULL + i], 4);
+      mbar_init(&bar[B_O_DONE + i], 1);
+    }
+    mbar_init(&bar[B_QPACK], 1);
+    mbar_init(&bar[B_QFULL], hasB ? 8 : 4);
+    mbar_init(&bar[B_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  if (warp < 8) {
+    regs_inc<SOFTMAX_REGS>();
+  } else {
+    regs_dec<PRODUCER_REGS>();
+  }
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int X = warp >> 2, wq = warp & 3;
+    if (X == 0 || hasB) {
+      const uint32_t row = tid & 127;
+      uint8_t* qtile = sm + (X ? Smem::QB : Smem::QA);
+      auto wait_all = [&](int b, uint32_t parity, uint32_t site) {
+        return __all_sync(0xffffffffu, mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site));
+      };
+      bool ok = wait_all(B_QPACK, 0, 0x4101);
+      if (ok) {
+        // widen this thread's packed Q row
+        const uint4* src = reinterpret_cast<const uint4*>(sm + Smem::QPK + X * 8192 + row * 64);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint4 c0, c1;
+          widen16(src[h], c0, c1);
+          *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h)) = c0;
+          *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h + 1)) = c1;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_QFULL]);
+        const int grow = (qt0 + X) * TILE + (int)row;
+        const float kq = __fmul_rn(a.sq[(size_t)bh * nblk + grow / QK_BLOCK], LOG2E / (SQRT_D * 256.0f));
+        const float* skb = a.sk + (size_t)bh * nblk;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t tS = tbase + X * 128 + lane_off, tO = tbase + 256 + X * 128 + lane_off;
+        const bool dbg_tile = dbg_run && (qt0 + X) == a.dbg_qt;
+        const int tail = P.N - (nt - 1) * TILE;   // valid keys in the last tile, 1..128
+        float m = -INFINITY, l = 0.0f;
+        float skn0 = __ldg(skb), skn1 = __ldg(skb + 1);
+        for (int j = 0; j < nt; ++j) {
+          const float sk0 = skn0, sk1 = skn1;
+          if (j + 1 < nt) {   // next tile's K scales, a tile ahead
+            skn0 = __ldg(skb + 2 * j + 2);
+            skn1 = __ldg(skb + 2 * j + 3);
+          }
+          // S_X(j) has landed -- and with it every earlier MMA, P.V(j-1) included
+          if (!(ok = wait_all(B_S_FULL + X, j & 1, 0x4102))) break;
+          tc_fence_after();
+          uint32_t s[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+          tmem_wait_ld();
+          const int nvalid = (j == nt - 1) ? tail : TILE;
+          if (nvalid < TILE) {
+#pragma unroll
+            for (int n = 0; n < 128; ++n)
+              if (n >= nvalid) s[n] = (uint32_t)S_PAD;
+          }
+          const float c0 = __fmul_rn(kq, sk0), c1 = __fmul_rn(kq, sk1);
+          // row max: floats 1.5*2^23 + 256 S are exact and ordered like S
+#pragma unroll
+          for (int n = 0; n < 128; ++n) s[n] += MAGIC_BITS;
+          float mh[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            mh[c] = fmax3(__int_as_float(s[16 * c]), __int_as_float(s[16 * c + 1]), __int_as_float(s[16 * c + 2]));
+#pragma unroll
+            for (int n = 3; n < 15; n += 2)
+              mh[c] = fmax3(mh[c], __int_as_float(s[16 * c + n]), __int_as_float(s[16 * c + n + 1]));
+            mh[c] = fmaxf(mh[c], __int_as_float(s[16 * c + 15]));
+          }
+          const float mx0 = fmaxf(fmax3(mh[0], mh[1], mh[2]), mh[3]);
+          const float mx1 = fmaxf(fmax3(mh[4], mh[5], mh[6]), mh[7]);
+          float tmax = __fmul_rn(mx0 - MAGIC, c0);
+          if (nvalid > 64) tmax = fmaxf(tmax, __fmul_rn(mx1 - MAGIC, c1));
+          const float m_new = fmaxf(m, tmax);
+          const bool moved = j > 0 && m_new > m;
+          const float alpha = moved ? ex2(m - m_new) : 1.0f;
+          // rows whose max moved: acc *= alpha (P.V(j-1) has landed)
+          if (__any_sync(0xffffffffu, moved)) {
+            const long long aq = __float2ll_rn(alpha * 1073741824.0f);   // round(2^30 alpha)
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t acc[16];
+              tmem_ld16(tO + 16 * c, acc);
+              tmem_wait_ld();
+              if (moved) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] = (uint32_t)(int)(((long long)(int)acc[e] * aq) >> 30);
+              }
+              tmem_st16(tO + 16 * c, acc);
+            }
+          }
+          m = m_new;
+          const float negm = -m;
+          uint32_t L = 0;
+          uint32_t pw[32];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {   // 8 keys per pair of words: evens, then odds
+            uint32_t wb[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int n = 4 * k + e;
+              const float x = fmaf(__int_as_float(s[n]) - MAGIC, n < 64 ? c0 : c1, negm);
+              wb[e] = __float_as_uint(fmaf(15.0f, ex2(x), MAGIC));   // low byte = w
+            }
+            const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
+            const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
+            pw[k] = __byte_perm(e02, e46, 0x5410);
+            pw[k + 1] = __byte_perm(o13, o57, 0x5410);
+            L = __dp4a(pw[k], 0x01010101u, L);
+            L = __dp4a(pw[k + 1], 0x01010101u, L);
+          }
+          if (nvalid < TILE) {   // keys past N leave the normaliser and the operand
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const uint32_t keep = p_word_mask(k, nvalid);
+              L -= __dp4a(pw[k] & ~keep, 0x01010101u, 0u);
+              pw[k] &= keep;
+            }
+          }
+          tmem_st32(tS + P_COL, pw);
+          l = fmaf(l, alpha, (float)L);
+          if (dbg_tile && j == a.dbg_kv) {
+#pragma unroll
+            for (int n = 0; n < 128; ++n) {
+              const int w = (int)((pw[2 * (n >> 3) + (n & 1)] >> (8 * ((n & 7) >> 1))) & 0xFF);
+              a.dbg_s[row * TILE + n] = n < nvalid ? ((int)(s[n] - MAGIC_BITS) >> 8) : 0;
+              a.dbg_p[row * TILE + n] = n < nvalid ? (int8_t)(w - 8) : (int8_t)-128;
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_P_FULL + X]);
+        }
+        if (ok) ok = wait_all(B_O_DONE + X, 0, 0x4105);
+        if (ok) {
+          // epilogue: O = acc * s_V / (16 l) -> fp16; loads are warp-collective,
+          // stores only for rows < N
+          tc_fence_after();
+          const float inv = 1.0f / (16.0f * l);
+          const float* svb = a.sv + (size_t)bh * D;
+          const bool store = grow < P.N && !dbg_run;
+          __half* orow = a.o + ((size_t)bh * P.N + (store ? grow : 0)) * D;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t acc[16];
+            tmem_ld16(tO + 16 * c, acc);
+            tmem_wait_ld();
+            uint32_t hv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float x0 = (float)(int)acc[2 * e] * __ldg(svb + 16 * c + 2 * e) * inv;
+              const float x1 = (float)(int)acc[2 * e + 1] * __ldg(svb + 16 * c + 2 * e + 1) * inv;
+              const __half2 h2 = __floats2half2_rn(x0, x1);
+              hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            if (store) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+              dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+              dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ widen INT4 -> INT8
+    const int wt = tid - 256, rsub = wt >> 2, h = wt & 3;
+    for (int j = 0; j < nt; ++j) {
+      const int st = j % PK_STAGES, s = j % OP_STAGES;
+      bool ok = mbar_wait_abortable(&bar[B_PK_FULL + st], (j / PK_STAGES) & 1, abort_flag, limit, err, 0x4401);
+      if (ok && j >= OP_STAGES)
+        ok = mbar_wait_abortable(&bar[B_OP_EMPTY + s], ((j / OP_STAGES) - 1) & 1, abort_flag, limit, err, 0x4402);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint8_t* src = sm + Smem::PK + st * 16384;
+      uint8_t* dst = sm + Smem::OP + s * 32768;
+#pragma unroll 4
+      for (int pass = 0; pass < 8; ++pass) {
+        const int r = pass * 32 + rsub;   // rows 0..127: K, 128..255: V^T
+        const uint4 u = *reinterpret_cast<const uint4*>(src + r * 64 + h * 16);
+        uint4 c0, c1;
+        widen16(u, c0, c1);
+        uint8_t* tile = dst + (r >> 7) * 16384;
+        *reinterpret_cast<uint4*>(tile + sw128_off(r & 127, 2 * h)) = c0;
+        *reinterpret_cast<uint4*>(tile + sw128_off(r & 127, 2 * h + 1)) = c1;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[B_OP_FULL + s]);
+        mbar_arrive(&bar[B_PK_EMPTY + st]);
+      }
+    }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------ bulk-copy producer
+    if (lane == 0) {
+      const uint8_t* qsrc = a.q4 + ((size_t)bh * P.N_pad + (size_t)qt0 * TILE) * (D / 2);
+      mbar_expect_tx(&bar[B_QPACK], hasB ? 16384u : 8192u);
+      bulk_g2s(sm + Smem::QPK, qsrc, 8192, &bar[B_QPACK]);
+      if (hasB) bulk_g2s(sm + Smem::QPK + 8192, qsrc + 8192, 8192, &bar[B_QPACK]);
+      const uint8_t* kb = a.k4 + (size_t)bh * P.N_pad * (D / 2);
+      const uint8_t* vb = a.v4t + (size_t)bh * P.N_pad * (D / 2);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % PK_STAGES;
+        if (j >= PK_STAGES && !mbar_wait_abortable(&bar[B_PK_EMPTY + st], ((j / PK_STAGES) - 1) & 1, abort_flag,
+                                                   limit, err, 0x4201))
+          break;
+        uint8_t* dst = sm + Smem::PK + st * 16384;
+        mbar_expect_tx(&bar[B_PK_FULL + st], 16384u);
+        bulk_g2s(dst, kb + (size_t)j * 8192, 8192, &bar[B_PK_FULL + st]);
+        bulk_g2s(dst + 8192, vb + (size_t)j * 8192, 8192, &bar[B_PK_FULL + st]);
+        issued = j + 1;
+      }
+      if (*abort_flag) {   // let every copy still in flight land before the CTA exits
+        mbar_wait(&bar[B_QPACK], 0, limit, err, 0x4203);
+        for (int j = issued > PK_STAGES ? issued - PK_STAGES : 0; j < issued; ++j)
+          mbar_wait(&bar[B_PK_FULL + j % PK_STAGES], (j / PK_STAGES) & 1, limit, err, 0x4204);
+      }
+    }
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t qa[2] = {smem_u32(sm + Smem::QA), smem_u32(sm + Smem::QB)};
+      const uint32_t op = smem_u32(sm + Smem::OP);
+      auto wait = [&](int b, uint32_t parity, uint32_t site) {
+        return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
+      };
+      auto issue_S = [&](int X, int j) {   // S_X(j) = Q_X K(j)^T
+        const uint32_t kt = op + (j % OP_STAGES) * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_i8(tbase + X * 128, sw128_desc(qa[X] + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, kk > 0);
+        umma_commit(&bar[B_S_FULL + X]);
+      };
+      auto issue_PV = [&](int X, int j) {   // O_X += W_X(j) V(j), W from TMEM
+        const uint32_t vt = op + (j % OP_STAGES) * 32768 + 16384;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_i8_tmem_a(tbase + 256 + X * 128, tbase + X * 128 + P_COL + 8 * kk, sw128_desc(vt + 32 * kk),
+                         IDESC_PV, (j > 0) || (kk > 0));
+      };
+      bool ok = wait(B_QFULL, 0, 0x4301) && wait(B_OP_FULL, 0, 0x4302);
+      if (ok) {
+        tc_fence_after();
+        issue_S(0, 0);
+        if (hasB) issue_S(1, 0);
+      }
+      for (int j = 1; j <= nt && ok; ++j) {
+        // tile j-1's P.V, then tile j's S, for A and then B
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (X == 1 && !hasB) break;
+          if (!(ok = wait(B_P_FULL + X, (j - 1) & 1, 0x4303 + X))) break;
+          tc_fence_after();
+          issue_PV(X, j - 1);
+          if (j < nt) {
+            if (!(ok = wait(B_OP_FULL + j % OP_STAGES, (j / OP_STAGES) & 1, 0x4305))) break;
+            tc_fence_after();
+            issue_S(X, j);
+          } else {
+            umma_commit(&bar[B_O_DONE + X]);
+          }
+        }
+        if (ok) umma_commit(&bar[B_OP_EMPTY + (j - 1) % OP_STAGES]);
+      }
+      // every MMA issued so far completes before TMEM is released
+      umma_commit(&bar[B_DRAIN]);
+      mbar_wait(&bar[B_DRAIN], 0, limit, err, 0x4308);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4t,
+                                  const float* sq, const float* sk, const float* sv, __half* o, void* ws, int dbg_bh,
+                                  int dbg_qtile, int dbg_kv, int32_t* dbg_s, int8_t* dbg_p, cudaStream_t st) {
+  const int smem = Smem::BYTES + 1024;   // > half the SM: one CTA per SM owns all 512 TMEM columns
+  cudaError_t e = cudaFuncSetAttribute(int4_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // The setmaxnreg split assumes the kernel launches with LAUNCH_REGS per
+  // thread; with fewer, the softmax warpgroups' increase could never be
+  // granted.  Refuse to launch rather than risk that.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, int4_attn_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+  KernelArgs a{p, q4, k4, v4t, sq, sk, sv, o, static_cast<WsHeader*>(ws), wait_limit(), dbg_bh, dbg_qtile, dbg_kv,
+               dbg_s, dbg_p};
+  const int n_qt = p.N_pad / TILE;
+  const dim3 grid = dbg_s ? dim3(1, 1) : dim3((n_qt + 1) / 2, p.BH);
+  int4_attn_kernel<<<grid, NUM_THREADS, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ra

@@ -76,8 +76,8 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
 cudaError_t launch_fp16_attention(const Prob& p, __half* o, void* ws, cudaStream_t st);
 cudaError_t launch_timeout_probe(void* ws, cudaStream_t st);
 
-// Iteration limit of every bounded device-side wait.
-uint32_t wait_limit();
+// Wall-clock limit (ns) of every bounded device-side wait.
+uint64_t wait_limit();
 
 // Host helpers shared with the allocation-free entry point (ra_noalloc.cu):
 // problem validation with derived sizes, and the coefficient table builder.

@@ -240,7 +240,9 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
     }
     w[t] = word;
   }
-  uint4* dst = reinterpret_cast<uint4*>(v4t + ((size_t)bh * D + c) * (P.N_pad / 2) + (size_t)blk * (QK_BLOCK / 2));
+  // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
+  uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
+                                        (size_t)(blk % 2) * (QK_BLOCK / 2));
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
   vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;

@@ -69,14 +69,60 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete, at most `limit`
-// polls.  Returns false (and records DEVERR_TIMEOUT) when the limit is hit.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit, DeviceErr* err,
+// Same, but the thread may sleep in hardware for up to `hint_ns` while the
+// phase is incomplete (woken early when it completes): no issue slots are
+// burnt spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint32_t kSleepHintNs = 10000;   // longest hardware sleep per poll
+
+// Waits for the phase with the given parity to complete, for at most
+// `limit_ns` of wall-clock time.  Returns false (and records DEVERR_TIMEOUT)
+// when the limit runs out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns, DeviceErr* err,
                                           uint32_t site) {
-  for (uint32_t it = 0; it < limit; ++it)
-    if (mbar_try_wait(bar, parity)) return true;
-  report(err, DEVERR_TIMEOUT, site);
-  return false;
+  if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, kSleepHintNs)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      report(err, DEVERR_TIMEOUT, site);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Waits as mbar_wait, but gives up at once when another role of the CTA has
+// set `abort_flag`, and sets it itself when its own limit runs out.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                    uint64_t limit_ns, DeviceErr* err, uint32_t site) {
+  if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (*abort_flag) return false;
+    if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      report(err, DEVERR_TIMEOUT, site);
+      return false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- bulk copy

@@ -164,14 +164,14 @@ def test_int4_path_is_deterministic(dev):
 def test_device_timeout_is_reported_not_hung(dev):
     cfg = SMALL["tiny"]
     ra = api.RotateAttention(cfg, dev, fp16_path=False)
-    api.debug_set_wait_limit(1)
+    api.debug_set_wait_timeout_us(1)
     try:
         api.debug_timeout_probe(ra.workspace)
         with pytest.raises(api.RotateAttnError) as e:
             ra.check()
         assert e.value.status == api.RA_ERR_DEVICE_TIMEOUT
     finally:
-        api.debug_set_wait_limit(0)
+        api.debug_set_wait_timeout_us(0)
     ra.check()          # cleared; the context is still usable
     q, k, v = synth.make_qkv(cfg)
     run_int4(cfg, dev, q, k, v)
