@@ -31,7 +31,7 @@
 // sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
 // The int32 P.V accumulator stays in TMEM across tiles; a row whose running
 // max moves rescales its accumulator in place with an integer multiply by
-// round(2^30 * exp(m_old - m_new)) (exp(...) is exactly 1 for every other
+// round(2^31 * exp(m_old - m_new)) (exp(...) is exactly 1 for every other
 // row).  The normaliser l is the running sum of w.
 //
 // INT4 codes are widened to 16*code (the nibble placed in the high half of
@@ -55,10 +55,12 @@ constexpr int NUM_THREADS = 512;
 constexpr int PK_STAGES = 3;   // packed K/V^T staging (bulk copies)
 constexpr int OP_STAGES = 4;   // widened K/V^T operands
 // Register split: launched at LAUNCH_REGS per thread (512 x 128 = 65536); the
-// widen and producer warpgroups drop to PRODUCER_REGS, the two softmax
-// warpgroups rise to SOFTMAX_REGS: 256 x 200 + 256 x 56 = 65536.
-constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 200, PRODUCER_REGS = 56;
-static_assert(256 * SOFTMAX_REGS + 256 * PRODUCER_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
+// widen warpgroup drops to WIDEN_REGS, the copy/MMA warpgroup to ISSUE_REGS,
+// the two softmax warpgroups rise to SOFTMAX_REGS:
+// 256 x 200 + 128 x 40 + 128 x 72 = 65536.
+constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 200, WIDEN_REGS = 40, ISSUE_REGS = 72;
+static_assert(256 * SOFTMAX_REGS + 128 * WIDEN_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS,
+              "register split");
 
 constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
 constexpr uint32_t IDESC_PV = make_idesc(2, 0, 1, 128, 128);   // s32 += u8 x s8
@@ -219,8 +221,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   const uint32_t tbase = *tslot;
   if (warp < 8) {
     regs_inc<SOFTMAX_REGS>();
+  } else if (warp < 12) {
+    regs_dec<WIDEN_REGS>();
   } else {
-    regs_dec<PRODUCER_REGS>();
+    regs_dec<ISSUE_REGS>();
   }
 
   if (warp < 8) {
@@ -269,6 +273,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
           tmem_wait_ld();
           const int nvalid = (j == nt - 1) ? tail : TILE;
+          if (dbg_tile && j == a.dbg_kv) {   // S = (256 S) >> 8, exactly
+#pragma unroll
+            for (int n = 0; n < 128; ++n) a.dbg_s[row * TILE + n] = n < nvalid ? ((int)s[n] >> 8) : 0;
+          }
           if (nvalid < TILE) {
 #pragma unroll
             for (int n = 0; n < 128; ++n)
@@ -294,40 +302,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const float m_new = fmaxf(m, tmax);
           const bool moved = j > 0 && m_new > m;
           const float alpha = moved ? ex2(m - m_new) : 1.0f;
-          // rows whose max moved: acc *= alpha (P.V(j-1) has landed)
-          if (__any_sync(0xffffffffu, moved)) {
-            const long long aq = __float2ll_rn(alpha * 1073741824.0f);   // round(2^30 alpha)
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-              uint32_t acc[16];
-              tmem_ld16(tO + 16 * c, acc);
-              tmem_wait_ld();
-              if (moved) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = (uint32_t)(int)(((long long)(int)acc[e] * aq) >> 30);
-              }
-              tmem_st16(tO + 16 * c, acc);
-            }
-          }
           m = m_new;
           const float negm = -m;
+          // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
+          // 64-key half whose largest x is below -5 holds only zero codes.
+          // Skip its exponentials when that is so for every row of the warp.
+          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < -5.0f),
+                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < -5.0f)};
           uint32_t L = 0;
           uint32_t pw[32];
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {   // 8 keys per pair of words: evens, then odds
-            uint32_t wb[8];
+          for (int h = 0; h < 2; ++h) {
+            if (zero_half[h]) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int n = 4 * k + e;
-              const float x = fmaf(__int_as_float(s[n]) - MAGIC, n < 64 ? c0 : c1, negm);
-              wb[e] = __float_as_uint(fmaf(15.0f, ex2(x), MAGIC));   // low byte = w
+              for (int k = 16 * h; k < 16 * h + 16; ++k) pw[k] = 0u;
+              continue;
             }
-            const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
-            const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
-            pw[k] = __byte_perm(e02, e46, 0x5410);
-            pw[k + 1] = __byte_perm(o13, o57, 0x5410);
-            L = __dp4a(pw[k], 0x01010101u, L);
-            L = __dp4a(pw[k + 1], 0x01010101u, L);
+#pragma unroll
+            for (int k = 16 * h; k < 16 * h + 16; k += 2) {   // 8 keys per pair of words: evens, then odds
+              uint32_t wb[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int n = 4 * k + e;
+                const float x = fmaf(__int_as_float(s[n]) - MAGIC, h ? c1 : c0, negm);
+                wb[e] = __float_as_uint(fmaf(15.0f, ex2(x), MAGIC));   // low byte = w
+              }
+              const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
+              const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
+              pw[k] = __byte_perm(e02, e46, 0x5410);
+              pw[k + 1] = __byte_perm(o13, o57, 0x5410);
+              L = __dp4a(pw[k], 0x01010101u, L);
+              L = __dp4a(pw[k + 1], 0x01010101u, L);
+            }
           }
           if (nvalid < TILE) {   // keys past N leave the normaliser and the operand
 #pragma unroll
@@ -339,11 +345,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           }
           tmem_st32(tS + P_COL, pw);
           l = fmaf(l, alpha, (float)L);
+          // rows whose max moved: acc *= alpha before P.V(j) adds to it (the
+          // arrival of S(j) means P.V(j-1) has landed)
+          if (__any_sync(0xffffffffu, moved)) {
+            // acc * alpha = (2 acc * round(2^31 alpha)) >> 32, |acc| < 2^28
+            const int aq = __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f));
+            uint32_t acc[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
+            tmem_wait_ld();
+            if (moved) {
+#pragma unroll
+              for (int e = 0; e < 128; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
+          }
           if (dbg_tile && j == a.dbg_kv) {
 #pragma unroll
             for (int n = 0; n < 128; ++n) {
               const int w = (int)((pw[2 * (n >> 3) + (n & 1)] >> (8 * ((n & 7) >> 1))) & 0xFF);
-              a.dbg_s[row * TILE + n] = n < nvalid ? ((int)(s[n] - MAGIC_BITS) >> 8) : 0;
               a.dbg_p[row * TILE + n] = n < nvalid ? (int8_t)(w - 8) : (int8_t)-128;
             }
           }
@@ -466,22 +487,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         issue_S(0, 0);
         if (hasB) issue_S(1, 0);
       }
-      for (int j = 1; j <= nt && ok; ++j) {
-        // tile j-1's P.V, then tile j's S, for A and then B
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (X == 1 && !hasB) break;
-          if (!(ok = wait(B_P_FULL + X, (j - 1) & 1, 0x4303 + X))) break;
+      // Serve whichever query tile has its P operand ready: tile X's step j
+      // is O_X += W_X(j-1) V(j-1) then S_X(j) (needs operand stage j).  An
+      // operand stage is released once both tiles have issued their P.V on it.
+      int next[2] = {1, hasB ? 1 : nt + 1};
+      int released = 0;
+      uint32_t idle = 0;
+      uint64_t t0 = 0;
+      while (ok && (next[0] <= nt || next[1] <= nt)) {
+        bool progress = false;
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          const int j = next[X];
+          if (j > nt || !mbar_test_wait(&bar[B_P_FULL + X], (j - 1) & 1)) continue;
+          if (j < nt && !mbar_test_wait(&bar[B_OP_FULL + j % OP_STAGES], (j / OP_STAGES) & 1)) continue;
           tc_fence_after();
           issue_PV(X, j - 1);
-          if (j < nt) {
-            if (!(ok = wait(B_OP_FULL + j % OP_STAGES, (j / OP_STAGES) & 1, 0x4305))) break;
-            tc_fence_after();
+          if (j < nt)
             issue_S(X, j);
-          } else {
+          else
             umma_commit(&bar[B_O_DONE + X]);
+          next[X] = j + 1;
+          progress = true;
+        }
+        const int done = min(next[0], next[1]) - 1;   // tiles whose P.V both tiles have issued
+        while (released < done && released < nt) {
+          umma_commit(&bar[B_OP_EMPTY + released % OP_STAGES]);
+          ++released;
+        }
+        if (progress) {
+          idle = 0;
+          t0 = 0;
+        } else if ((++idle & 63u) != 0) {
+          __nanosleep(20);
+        } else {
+          if (*abort_flag) {
+            ok = false;
+          } else {
+            const uint64_t t = globaltimer_ns();
+            if (t0 == 0) {
+              t0 = t;
+            } else if (t - t0 > limit) {
+              *abort_flag = 1;
+              report(err, DEVERR_TIMEOUT, 0x4303);
+              ok = false;
+            }
           }
         }
-        if (ok) umma_commit(&bar[B_OP_EMPTY + (j - 1) % OP_STAGES]);
       }
       // every MMA issued so far completes before TMEM is released
       umma_commit(&bar[B_DRAIN]);
