@@ -14,17 +14,25 @@
 //   WG2 (warps 8-11)   widen packed INT4 K and V^T tiles into INT8 (16*code)
 //                      in 128-byte-swizzled K-major SMEM operands, 4 stages
 //   WG3 warp 12        bulk-copy producer (packed K, V^T tiles, 8 KB each,
-//                      into a 3-stage ring; the two packed Q tiles once)
-//       warp 13        TMEM owner and single-thread tcgen05.mma issuer
+//                      into a 3-stage ring)
+//       warps 13, 14   MMA issuers, one thread per query tile (warp 13 also
+//                      owns the TMEM allocation)
+//       warp 15        writes the constant bf16 operand at start-up
 // TMEM (512 columns): S_A | S_B | O_A | O_B, 128 int32 columns each.  The P
 // operand of a tile (128 rows x 128 u8 = 32 columns) is stored by the softmax
 // threads into the last 32 columns of their own S region once S is in
 // registers, and read from there by the P.V MMA (A operand in TMEM).
 // MMA order per query tile X: S_X(0); then for every tile j: O_X += W_X(j)
-// V(j), S_X(j+1) -- tiles A and B interleaved, so the tensor core runs one
-// tile's MMAs while the other tile's softmax runs (ping-pong).  Because the
-// MMAs of one CTA complete in issue order, the arrival of S_X(j+1) also means
-// that P.V(j) has landed: the softmax may rescale O_X right then.
+// V(j), S_X(j+1).  Each tile has its own issuing thread, blocked on that
+// tile's barriers, so the tensor core runs one tile's MMAs while the other
+// tile's softmax runs (ping-pong) with no polling between them.  Because the
+// MMAs of one thread complete in issue order, the arrival of S_X(j+1) also
+// means that P.V(j) has landed: the softmax may rescale O_X right then.
+//
+// S_X(j) starts as 1.5 * 2^23 in every accumulator (one bf16 MMA with a
+// constant operand), so after the integer MMAs add 256 S the accumulator bits
+// are exactly the float 1.5 * 2^23 + 256 S: the softmax takes its row max and
+// its exponent arguments on the raw bits, with no integer-to-float step.
 //
 // The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15], fed as an
 // unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
@@ -64,6 +72,7 @@ static_assert(256 * SOFTMAX_REGS + 128 * WIDEN_REGS + 128 * ISSUE_REGS <= NUM_TH
 
 constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
 constexpr uint32_t IDESC_PV = make_idesc(2, 0, 1, 128, 128);   // s32 += u8 x s8
+constexpr uint32_t IDESC_INIT = make_idesc(1, 1, 1, 128, 128);  // f32 = bf16 x bf16
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float SQRT_D = 11.313708498984761f;
 constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
@@ -75,14 +84,14 @@ struct Smem {
   static constexpr uint32_t QA = 0, QB = 16384;   // widened Q tiles
   static constexpr uint32_t OP = 32768;           // 4 x 32 KB: widened K (+0), V^T (+16 KB)
   static constexpr uint32_t PK = 163840;          // 3 x 16 KB: packed K (+0), V^T (+8 KB)
-  static constexpr uint32_t QPK = 212992;         // 16 KB: packed Q staging
-  static constexpr uint32_t BAR = 229376;
+  static constexpr uint32_t CT = 212992;          // 4 KB: bf16 operand that sets S to 1.5 * 2^23
+  static constexpr uint32_t BAR = 217088;
   static constexpr uint32_t BYTES = BAR + 256;
 };
 
 enum : int {
-  B_PK_FULL = 0, B_PK_EMPTY = 3, B_OP_FULL = 6, B_OP_EMPTY = 10, B_QPACK = 14, B_QFULL = 15,
-  B_S_FULL = 16, B_P_FULL = 18, B_O_DONE = 20, B_DRAIN = 22, NBAR = 23
+  B_PK_FULL = 0, B_PK_EMPTY = 3, B_OP_FULL = 6, B_OP_EMPTY = 10, B_QFULL = 14,
+  B_S_FULL = 15, B_P_FULL = 17, B_O_DONE = 19, B_DRAIN = 21, NBAR = 23
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -137,6 +146,14 @@ __device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
       "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// K-major operand without swizzle: 8-row x 16-byte core matrices, rows 16
+// bytes apart; 8-row groups 128 bytes apart (stride byte offset), the two
+// 8-element K halves 2048 bytes apart (leading byte offset); K = 16 bf16.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(2048u >> 4) << 16) | ((uint64_t)(128u >> 4) << 32) |
+         ((uint64_t)1u << 46);
 }
 
 // 4 packed words (32 codes) -> two 16-byte chunks of 16*code, evens then odds
@@ -198,22 +215,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
     }
     for (int i = 0; i < OP_STAGES; ++i) {
       mbar_init(&bar[B_OP_FULL + i], 4);
-      mbar_init(&bar[B_OP_EMPTY + i], 1);
+      mbar_init(&bar[B_OP_EMPTY + i], hasB ? 2 : 1);   // one commit per query tile's MMA thread
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[B_S_FULL + i], 1);
       mbar_init(&bar[B_P_FULL + i], 4);
       mbar_init(&bar[B_O_DONE + i], 1);
+      mbar_init(&bar[B_DRAIN + i], 1);
     }
-    mbar_init(&bar[B_QPACK], 1);
     mbar_init(&bar[B_QFULL], hasB ? 8 : 4);
-    mbar_init(&bar[B_DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 13) {
     tmem_alloc(tslot, 512);
     tmem_relinquish();
+  }
+  if (warp == 15) {
+    // bf16 2048 in columns 0..2 of every row, zero elsewhere: used as both
+    // operands, A B^T = 3 * 2048^2 = 1.5 * 2^23 in every accumulator, whose
+    // bits 0x4B400000 the integer S MMAs then add 256 S to
+    uint32_t* ct = reinterpret_cast<uint32_t*>(sm + Smem::CT);
+    for (int i = lane; i < 1024; i += 32) {
+      const int w = i & 3;   // row i / 4 holds K elements 0..7 in bytes 16 r .. 16 r + 15
+      ct[i] = i >= 512 ? 0u : (w == 0 ? 0x45004500u : (w == 1 ? 0x00004500u : 0u));
+    }
+    fence_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -236,14 +263,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       auto wait_all = [&](int b, uint32_t parity, uint32_t site) {
         return __all_sync(0xffffffffu, mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site));
       };
-      bool ok = wait_all(B_QPACK, 0, 0x4101);
-      if (ok) {
+      bool ok = true;
+      {
         // widen this thread's packed Q row
-        const uint4* src = reinterpret_cast<const uint4*>(sm + Smem::QPK + X * 8192 + row * 64);
+        const uint4* src = reinterpret_cast<const uint4*>(a.q4 + ((size_t)bh * P.N_pad + (size_t)(qt0 + X) * TILE + row) * (D / 2));
+        uint4 qp[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) qp[h] = __ldg(src + h);
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           uint4 c0, c1;
-          widen16(src[h], c0, c1);
+          widen16(qp[h], c0, c1);
           *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h)) = c0;
           *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h + 1)) = c1;
         }
@@ -275,17 +305,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const int nvalid = (j == nt - 1) ? tail : TILE;
           if (dbg_tile && j == a.dbg_kv) {   // S = (256 S) >> 8, exactly
 #pragma unroll
-            for (int n = 0; n < 128; ++n) a.dbg_s[row * TILE + n] = n < nvalid ? ((int)s[n] >> 8) : 0;
+            for (int n = 0; n < 128; ++n) a.dbg_s[row * TILE + n] = n < nvalid ? ((int)(s[n] - MAGIC_BITS) >> 8) : 0;
           }
           if (nvalid < TILE) {
 #pragma unroll
             for (int n = 0; n < 128; ++n)
-              if (n >= nvalid) s[n] = (uint32_t)S_PAD;
+              if (n >= nvalid) s[n] = (uint32_t)(MAGIC_BITS + S_PAD);
           }
           const float c0 = __fmul_rn(kq, sk0), c1 = __fmul_rn(kq, sk1);
-          // row max: floats 1.5*2^23 + 256 S are exact and ordered like S
-#pragma unroll
-          for (int n = 0; n < 128; ++n) s[n] += MAGIC_BITS;
+          // row max: the accumulators hold the bits of the floats 1.5*2^23 +
+          // 256 S, exact and ordered like S
           float mh[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -307,8 +336,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
           // 64-key half whose largest x is below -5 holds only zero codes.
           // Skip its exponentials when that is so for every row of the warp.
-          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < -5.0f),
-                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < -5.0f)};
+          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < -5.0f) != 0,
+                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < -5.0f) != 0};
           uint32_t L = 0;
           uint32_t pw[32];
 #pragma unroll
@@ -435,10 +464,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   } else if (warp == 12) {
     // ------------------------------------------------------------ bulk-copy producer
     if (lane == 0) {
-      const uint8_t* qsrc = a.q4 + ((size_t)bh * P.N_pad + (size_t)qt0 * TILE) * (D / 2);
-      mbar_expect_tx(&bar[B_QPACK], hasB ? 16384u : 8192u);
-      bulk_g2s(sm + Smem::QPK, qsrc, 8192, &bar[B_QPACK]);
-      if (hasB) bulk_g2s(sm + Smem::QPK + 8192, qsrc + 8192, 8192, &bar[B_QPACK]);
       const uint8_t* kb = a.k4 + (size_t)bh * P.N_pad * (D / 2);
       const uint8_t* vb = a.v4t + (size_t)bh * P.N_pad * (D / 2);
       int issued = 0;
@@ -454,90 +479,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         issued = j + 1;
       }
       if (*abort_flag) {   // let every copy still in flight land before the CTA exits
-        mbar_wait(&bar[B_QPACK], 0, limit, err, 0x4203);
         for (int j = issued > PK_STAGES ? issued - PK_STAGES : 0; j < issued; ++j)
           mbar_wait(&bar[B_PK_FULL + j % PK_STAGES], (j / PK_STAGES) & 1, limit, err, 0x4204);
       }
     }
-  } else if (warp == 13) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t qa[2] = {smem_u32(sm + Smem::QA), smem_u32(sm + Smem::QB)};
+  } else if (warp == 13 || warp == 14) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread per query tile, each blocked on its own tile's barriers, so
+    // each tile's MMAs go out as soon as its P operand is stored.  Tile X's
+    // step j is O_X += W_X(j-1) V(j-1), then S_X(j) = Q_X K(j)^T (operand
+    // stage j).  MMAs of one thread complete in issue order; the two threads'
+    // MMAs touch disjoint TMEM and only read the shared operand stages, whose
+    // release counts one commit from each thread.
+    const int X = warp - 13;
+    if (lane == 0 && (X == 0 || hasB)) {
+      const uint32_t qa = smem_u32(sm + (X ? Smem::QB : Smem::QA));
       const uint32_t op = smem_u32(sm + Smem::OP);
+      const uint64_t dc = plain_desc(smem_u32(sm + Smem::CT));
+      const uint32_t tS = tbase + X * 128, tO = tbase + 256 + X * 128;
       auto wait = [&](int b, uint32_t parity, uint32_t site) {
         return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
       };
-      auto issue_S = [&](int X, int j) {   // S_X(j) = Q_X K(j)^T
-        const uint32_t kt = op + (j % OP_STAGES) * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_i8(tbase + X * 128, sw128_desc(qa[X] + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, kk > 0);
-        umma_commit(&bar[B_S_FULL + X]);
-      };
-      auto issue_PV = [&](int X, int j) {   // O_X += W_X(j) V(j), W from TMEM
-        const uint32_t vt = op + (j % OP_STAGES) * 32768 + 16384;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_i8_tmem_a(tbase + 256 + X * 128, tbase + X * 128 + P_COL + 8 * kk, sw128_desc(vt + 32 * kk),
-                         IDESC_PV, (j > 0) || (kk > 0));
-      };
-      bool ok = wait(B_QFULL, 0, 0x4301) && wait(B_OP_FULL, 0, 0x4302);
-      if (ok) {
+      bool ok = wait(B_QFULL, 0, 0x4301);
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (j > 0 && !(ok = wait(B_P_FULL + X, (j - 1) & 1, 0x4302))) break;
+        if (j < nt && !(ok = wait(B_OP_FULL + j % OP_STAGES, (j / OP_STAGES) & 1, 0x4303))) break;
         tc_fence_after();
-        issue_S(0, 0);
-        if (hasB) issue_S(1, 0);
-      }
-      // Serve whichever query tile has its P operand ready: tile X's step j
-      // is O_X += W_X(j-1) V(j-1) then S_X(j) (needs operand stage j).  An
-      // operand stage is released once both tiles have issued their P.V on it.
-      int next[2] = {1, hasB ? 1 : nt + 1};
-      int released = 0;
-      uint32_t idle = 0;
-      uint64_t t0 = 0;
-      while (ok && (next[0] <= nt || next[1] <= nt)) {
-        bool progress = false;
+        if (j > 0) {   // O_X += W_X(j-1) V(j-1), W from TMEM
+          const uint32_t vt = op + ((j - 1) % OP_STAGES) * 32768 + 16384;
 #pragma unroll
-        for (int X = 0; X < 2; ++X) {
-          const int j = next[X];
-          if (j > nt || !mbar_test_wait(&bar[B_P_FULL + X], (j - 1) & 1)) continue;
-          if (j < nt && !mbar_test_wait(&bar[B_OP_FULL + j % OP_STAGES], (j / OP_STAGES) & 1)) continue;
-          tc_fence_after();
-          issue_PV(X, j - 1);
-          if (j < nt)
-            issue_S(X, j);
-          else
-            umma_commit(&bar[B_O_DONE + X]);
-          next[X] = j + 1;
-          progress = true;
+          for (int kk = 0; kk < 4; ++kk)
+            umma_i8_tmem_a(tO, tS + P_COL + 8 * kk, sw128_desc(vt + 32 * kk), IDESC_PV, (j > 1) || (kk > 0));
+          umma_commit(&bar[B_OP_EMPTY + (j - 1) % OP_STAGES]);
         }
-        const int done = min(next[0], next[1]) - 1;   // tiles whose P.V both tiles have issued
-        while (released < done && released < nt) {
-          umma_commit(&bar[B_OP_EMPTY + released % OP_STAGES]);
-          ++released;
-        }
-        if (progress) {
-          idle = 0;
-          t0 = 0;
-        } else if ((++idle & 63u) != 0) {
-          __nanosleep(20);
+        if (j < nt) {   // S_X(j): set to 1.5 * 2^23, then += 256 Q_X K(j)^T
+          const uint32_t kt = op + (j % OP_STAGES) * 32768;
+          umma_f16(tS, dc, dc, IDESC_INIT, 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, 1);
+          umma_commit(&bar[B_S_FULL + X]);
         } else {
-          if (*abort_flag) {
-            ok = false;
-          } else {
-            const uint64_t t = globaltimer_ns();
-            if (t0 == 0) {
-              t0 = t;
-            } else if (t - t0 > limit) {
-              *abort_flag = 1;
-              report(err, DEVERR_TIMEOUT, 0x4303);
-              ok = false;
-            }
-          }
+          umma_commit(&bar[B_O_DONE + X]);
         }
       }
-      // every MMA issued so far completes before TMEM is released
-      umma_commit(&bar[B_DRAIN]);
-      mbar_wait(&bar[B_DRAIN], 0, limit, err, 0x4308);
+      // every MMA this thread issued completes before TMEM is released
+      umma_commit(&bar[B_DRAIN + X]);
+      mbar_wait(&bar[B_DRAIN + X], 0, limit, err, 0x4308);
     }
   }
 
