@@ -34,7 +34,7 @@ from int4_quantized_attention_b200 import synth  # noqa: E402
 from int4_quantized_attention_b200.schedule import BENCH_SCHEDULE  # noqa: E402
 
 METRIC = "INT4 attention TOPS (4*N^2*d*H/time) and fraction of B200 INT8 tensor peak"
-KERNELS_PER_STEP = 4      # qk_quant, v_amax, v_quant, int4_attn
+KERNELS_PER_STEP = 5      # qk_quant, v_amax, v_quant, expand, int4_attn
 # Nominal dense tensor rates: int8 (= fp8) is twice bf16/fp16 on B200.
 INT8_PER_BF16 = 2.0
 
@@ -267,7 +267,7 @@ def our_arm(args, cfg, rank, world):
         "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
                    "grid": [cfg.F, cfg.Hh, cfg.W], "n_text": cfg.n_text, "split": list(cfg.split),
                    "rotation": cfg.rot, "parallelism": "replicas" if world > 1 else "single-gpu",
-                   "l2": "inputs larger than L2 (q,k,v 2.3 GB; packed K/V 0.39 GB per pass)"},
+                   "l2": "inputs larger than L2 (q,k,v 2.3 GB; INT8 K/V operand images 0.77 GB per pass)"},
         "roofline": {"kernel": "int4_attn_kernel", "bound": "tensor", "achieved": attn_tops,
                      "peak": peak_int8, "unit": "TOPS", "frac": attn_tops / peak_int8, "traffic": profiled_traffic(cfg),
                      "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TF/s x 2 (int8:bf16 nominal "

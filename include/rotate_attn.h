@@ -97,9 +97,12 @@ ra_status ra_validate(const ra_problem *p);
 size_t ra_qkv4_bytes(const ra_problem *p);
 ra_status ra_qkv4_bind(const ra_problem *p, void *base, size_t bytes, ra_qkv4 *out);
 
-/* Workspace: error word, RoPE/rotation tables, V channel-amax scratch and,
- * when with_fp16_path != 0, the FP16 path's position-encoded Q, K and
- * transposed V (3 * B*H*N_pad*128 fp16).  Device memory owned by the caller. */
+/* Workspace: error word, RoPE/rotation tables, V channel-amax scratch (all
+ * the prologue needs); the INT4 attention's INT8 operand images of Q, K and
+ * V^T, which ra_int4_attention_fwd expands from the packed codes on every
+ * call (3 * B*H*N_pad*128 bytes); and, when with_fp16_path != 0, the FP16
+ * path's position-encoded Q, K and transposed V (3 * B*H*N_pad*128 fp16).
+ * Device memory owned by the caller. */
 size_t ra_workspace_bytes(const ra_problem *p, int with_fp16_path);
 
 /* Builds the RoPE/rotation coefficient tables on the host (float64 libm,
@@ -119,10 +122,12 @@ ra_status ra_rotate_quantize_qkv(const ra_problem *p, const void *q, const void 
                                  const ra_qkv4 *out, void *workspace, size_t workspace_bytes,
                                  ra_stream stream);
 
-/* INT4 attention forward: S = Q K^T on INT8 tensor cores (INT4 codes widened
- * to INT8), online softmax over 128-key tiles, P = exp(s - m) quantised to
+/* INT4 attention forward: S = Q K^T on INT8 tensor cores (the INT4 codes
+ * are first expanded to INT8 operand images in the workspace, two launches
+ * per call), online softmax over 128-key tiles, P = exp(s - m) quantised to
  * rne(15 P) - 8, P.V with the zero-point correction, fp16 output.
  * in: from ra_rotate_quantize_qkv; o: fp16 [B][H][N][128].
+ * Workspace: ra_workspace_bytes(p, 0) bytes at least.
  * (Abstract; Sec. 4.2 as summarised in the referee report and ledger.) */
 ra_status ra_int4_attention_fwd(const ra_problem *p, const ra_qkv4 *in, void *o,
                                 void *workspace, size_t workspace_bytes, ra_stream stream);

@@ -145,10 +145,12 @@ QkvLayout qkv_layout(const ra::Prob& P) {
   return L;
 }
 
-ra_status check_ws(const ra::Prob& P, const void* ws, size_t bytes, bool fp16) {
+enum class WsUse { prologue, int4, fp16 };
+
+ra_status check_ws(const ra::Prob& P, const void* ws, size_t bytes, WsUse use) {
   if (!aligned16(ws)) return fail(RA_ERR_INVALID_ARG, "workspace pointer NULL or not 16-byte aligned");
   const ra::WsLayout L = ra::ws_layout(P);
-  const size_t need = fp16 ? L.total_fp16 : L.base_bytes;
+  const size_t need = use == WsUse::fp16 ? L.total_fp16 : (use == WsUse::int4 ? L.base_bytes : L.pro_bytes);
   if (bytes < need) return fail(RA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", bytes, need);
   return RA_OK;
 }
@@ -240,7 +242,7 @@ ra_status ra_prepare(const ra_problem* p, void* ws, size_t ws_bytes, ra_stream s
   ra::Prob P;
   ra_status st = derive(p, &P);
   if (st != RA_OK) return st;
-  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, WsUse::prologue)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const ra::WsLayout L = ra::ws_layout(P);
   std::vector<float> tab(4 * (size_t)P.n_tab);
@@ -266,7 +268,7 @@ ra_status ra_rotate_quantize_qkv(const ra_problem* p, const void* q, const void*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v))
     return fail(RA_ERR_INVALID_ARG, "q, k or v NULL or not 16-byte aligned");
   if ((st = check_qkv4(out)) != RA_OK) return st;
-  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, WsUse::prologue)) != RA_OK) return st;
   cudaError_t e = ra::launch_prologue(P, static_cast<const __half*>(q), static_cast<const __half*>(k),
                                       static_cast<const __half*>(v), out->q4, out->k4, out->v4t, out->sq, out->sk,
                                       out->sv, out->vsum, ws, static_cast<cudaStream_t>(stream));
@@ -280,7 +282,7 @@ ra_status ra_int4_attention_fwd(const ra_problem* p, const ra_qkv4* in, void* o,
   if (st != RA_OK) return st;
   if ((st = check_qkv4(in)) != RA_OK) return st;
   if (!aligned16(o)) return fail(RA_ERR_INVALID_ARG, "output NULL or not 16-byte aligned");
-  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, WsUse::int4)) != RA_OK) return st;
   cudaError_t e = ra::launch_int4_attention(P, in->q4, in->k4, in->v4t, in->sq, in->sk, in->sv,
                                             static_cast<__half*>(o), ws, -1, -1, -1, nullptr, nullptr,
                                             static_cast<cudaStream_t>(stream));
@@ -294,7 +296,7 @@ ra_status ra_fp16_attention_fwd(const ra_problem* p, const void* q, const void* 
   if (st != RA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(RA_ERR_INVALID_ARG, "q, k, v or o NULL or not 16-byte aligned");
-  if ((st = check_ws(P, ws, ws_bytes, true)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, WsUse::fp16)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = ra::launch_fp16_prologue(P, static_cast<const __half*>(q), static_cast<const __half*>(k),
                                            static_cast<const __half*>(v), ws, s);
@@ -341,7 +343,7 @@ ra_status ra_debug_int4_tile(const ra_problem* p, const ra_qkv4* in, int bh, int
   ra_status st = derive(p, &P);
   if (st != RA_OK) return st;
   if ((st = check_qkv4(in)) != RA_OK) return st;
-  if ((st = check_ws(P, ws, ws_bytes, false)) != RA_OK) return st;
+  if ((st = check_ws(P, ws, ws_bytes, WsUse::int4)) != RA_OK) return st;
   if (bh < 0 || bh >= P.BH || q_tile < 0 || q_tile >= P.N_pad / ra::TILE || kv_tile < 0 ||
       kv_tile >= P.N_pad / ra::TILE)
     return fail(RA_ERR_INVALID_ARG, "debug tile index out of range");

@@ -11,13 +11,17 @@
 // threads in four warpgroups:
 //   WG0 (warps 0-3)    softmax of tile A, thread t = query row t = TMEM lane t
 //   WG1 (warps 4-7)    softmax of tile B
-//   WG2 (warps 8-11)   widen packed INT4 K and V^T tiles into INT8 (16*code)
-//                      in 128-byte-swizzled K-major SMEM operands, 4 stages
-//   WG3 warp 12        bulk-copy producer (packed K, V^T tiles, 8 KB each,
-//                      into a 3-stage ring)
+//   WG2 (warps 8-11)   O correction: rescales the accumulator rows whose max
+//                      moved, for both tiles, off the softmax warps' path
+//   WG3 warp 12        bulk-copy producer: the two Q operand tiles once, then
+//                      the K and V^T operand tiles (16 KB each) into a
+//                      5-stage ring
 //       warps 13, 14   MMA issuers, one thread per query tile (warp 13 also
 //                      owns the TMEM allocation)
 //       warp 15        writes the constant bf16 operand at start-up
+// The packed INT4 inputs are expanded once per call, by expand_kernel, into
+// INT8 operand images laid out exactly as the MMAs read them from SMEM, so
+// the attention kernel itself only copies tiles.
 // TMEM (512 columns): S_A | S_B | O_A | O_B, 128 int32 columns each.  The P
 // operand of a tile (128 rows x 128 u8 = 32 columns) is stored by the softmax
 // threads into the last 32 columns of their own S region once S is in
@@ -27,7 +31,9 @@
 // tile's barriers, so the tensor core runs one tile's MMAs while the other
 // tile's softmax runs (ping-pong) with no polling between them.  Because the
 // MMAs of one thread complete in issue order, the arrival of S_X(j+1) also
-// means that P.V(j) has landed: the softmax may rescale O_X right then.
+// means that P.V(j) has landed: O_X may be rescaled right then, and must be
+// before P.V(j+1), whose issue waits for the correction warps as well as for
+// the softmax warps.
 //
 // S_X(j) starts as 1.5 * 2^23 in every accumulator (one bf16 MMA with a
 // constant operand), so after the integer MMAs add 256 S the accumulator bits
@@ -38,13 +44,13 @@
 // unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
 // sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
 // The int32 P.V accumulator stays in TMEM across tiles; a row whose running
-// max moves rescales its accumulator in place with an integer multiply by
+// max moves has its accumulator rescaled in place with an integer multiply by
 // round(2^31 * exp(m_old - m_new)) (exp(...) is exactly 1 for every other
 // row).  The normaliser l is the running sum of w.
 //
-// INT4 codes are widened to 16*code (the nibble placed in the high half of
+// INT4 codes are expanded to 16*code (the nibble placed in the high half of
 // the byte), so S comes out as 256*S and P.V as 16*P.V, exactly; both factors
-// fold into the dequantisation.  Within every 8-element group the widened
+// fold into the dequantisation.  Within every 8-element group the expanded
 // operands hold even elements first, then odd ones (channels for Q and K,
 // keys for V^T); the P operand is packed in the same key order.
 //
@@ -60,14 +66,13 @@ namespace ra {
 namespace {
 
 constexpr int NUM_THREADS = 512;
-constexpr int PK_STAGES = 3;   // packed K/V^T staging (bulk copies)
-constexpr int OP_STAGES = 4;   // widened K/V^T operands
+constexpr int OP_STAGES = 5;   // INT8 K / V^T operand tiles (bulk copies)
 // Register split: launched at LAUNCH_REGS per thread (512 x 128 = 65536); the
-// widen warpgroup drops to WIDEN_REGS, the copy/MMA warpgroup to ISSUE_REGS,
-// the two softmax warpgroups rise to SOFTMAX_REGS:
-// 256 x 200 + 128 x 40 + 128 x 72 = 65536.
-constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 200, WIDEN_REGS = 40, ISSUE_REGS = 72;
-static_assert(256 * SOFTMAX_REGS + 128 * WIDEN_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS,
+// correction warpgroup drops to CORR_REGS, the copy/MMA warpgroup to
+// ISSUE_REGS, the two softmax warpgroups rise to SOFTMAX_REGS:
+// 256 x 192 + 128 x 64 + 128 x 64 = 65536.
+constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 192, CORR_REGS = 64, ISSUE_REGS = 64;
+static_assert(256 * SOFTMAX_REGS + 128 * CORR_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS,
               "register split");
 
 constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
@@ -81,18 +86,19 @@ constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6), still e
 constexpr uint32_t P_COL = 96;    // P operand: columns 96..127 of the tile's S region
 
 struct Smem {
-  static constexpr uint32_t QA = 0, QB = 16384;   // widened Q tiles
-  static constexpr uint32_t OP = 32768;           // 4 x 32 KB: widened K (+0), V^T (+16 KB)
-  static constexpr uint32_t PK = 163840;          // 3 x 16 KB: packed K (+0), V^T (+8 KB)
-  static constexpr uint32_t CT = 212992;          // 4 KB: bf16 operand that sets S to 1.5 * 2^23
-  static constexpr uint32_t BAR = 217088;
-  static constexpr uint32_t BYTES = BAR + 256;
+  static constexpr uint32_t QA = 0, QB = 16384;   // INT8 Q operand tiles
+  static constexpr uint32_t OP = 32768;           // 5 x 32 KB: INT8 K (+0), V^T (+16 KB)
+  static constexpr uint32_t CT = 196608;          // 4 KB: bf16 operand that sets S to 1.5 * 2^23
+  static constexpr uint32_t CQ = 200704;          // 2 x 128 ints: per-row O rescale factors
+  static constexpr uint32_t BAR = 201728;
+  static constexpr uint32_t BYTES = BAR + 512;
 };
 
 enum : int {
-  B_PK_FULL = 0, B_PK_EMPTY = 3, B_OP_FULL = 6, B_OP_EMPTY = 10, B_QFULL = 14,
-  B_S_FULL = 15, B_P_FULL = 17, B_O_DONE = 19, B_DRAIN = 21, NBAR = 23
+  B_OP_FULL = 0, B_OP_EMPTY = 5, B_QFULL = 10, B_S_FULL = 11, B_P_FULL = 13, B_O_DONE = 15, B_DRAIN = 17,
+  B_CREQ = 19, NBAR = 27
 };
+constexpr int NO_RESCALE = -1;   // rescale factor of a row whose max stayed
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -175,11 +181,36 @@ __device__ __forceinline__ uint32_t p_word_mask(int k, int nvalid) {
   return m;
 }
 
+// INT4 -> INT8 operand images: one thread per 16 packed bytes (32 codes of
+// one row).  Q and K rows are tokens, V^T rows are channels (its tiles are
+// already 128 keys wide); row r of 128-row tile t lands, as 16 * code with
+// even then odd elements of every 8-group, 128-byte swizzled at
+// image + (b*H + h, t) * 16 KB.  The image of a tile is the SMEM operand of
+// the MMA byte for byte.
+__global__ void __launch_bounds__(256) expand_kernel(const uint8_t* __restrict__ q4, const uint8_t* __restrict__ k4,
+                                                     const uint8_t* __restrict__ v4t, uint8_t* __restrict__ qimg,
+                                                     uint8_t* __restrict__ kimg, uint8_t* __restrict__ vimg,
+                                                     size_t units) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= units) return;
+  const int which = blockIdx.y;
+  const uint8_t* src = which == 0 ? q4 : (which == 1 ? k4 : v4t);
+  uint8_t* dst = which == 0 ? qimg : (which == 1 ? kimg : vimg);
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(src) + i);
+  const size_t grow = i >> 2;   // (b*H + h) * N_pad + 128 t + r
+  const uint32_t h = (uint32_t)(i & 3), r = (uint32_t)(grow & 127);
+  uint8_t* tile = dst + (grow >> 7) * 16384;
+  uint4 c0, c1;
+  widen16(u, c0, c1);
+  *reinterpret_cast<uint4*>(tile + sw128_off(r, 2 * h)) = c0;
+  *reinterpret_cast<uint4*>(tile + sw128_off(r, 2 * h + 1)) = c1;
+}
+
 struct KernelArgs {
   Prob P;
-  const uint8_t* q4;
-  const uint8_t* k4;
-  const uint8_t* v4t;
+  const uint8_t* qimg;   // INT8 operand images [BH][N_pad / 128][16 KB]
+  const uint8_t* kimg;
+  const uint8_t* vimg;
   const float* sq;
   const float* sk;
   const float* sv;
@@ -209,21 +240,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   const uint64_t limit = a.limit;
 
   if (tid == 0) {
-    for (int i = 0; i < PK_STAGES; ++i) {
-      mbar_init(&bar[B_PK_FULL + i], 1);
-      mbar_init(&bar[B_PK_EMPTY + i], 4);
-    }
     for (int i = 0; i < OP_STAGES; ++i) {
-      mbar_init(&bar[B_OP_FULL + i], 4);
+      mbar_init(&bar[B_OP_FULL + i], 1);
       mbar_init(&bar[B_OP_EMPTY + i], hasB ? 2 : 1);   // one commit per query tile's MMA thread
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[B_S_FULL + i], 1);
-      mbar_init(&bar[B_P_FULL + i], 4);
+      mbar_init(&bar[B_P_FULL + i], 8);   // 4 softmax warps + 4 correction warps
       mbar_init(&bar[B_O_DONE + i], 1);
       mbar_init(&bar[B_DRAIN + i], 1);
     }
-    mbar_init(&bar[B_QFULL], hasB ? 8 : 4);
+    mbar_init(&bar[B_QFULL], 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&bar[B_CREQ + i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -249,7 +277,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   if (warp < 8) {
     regs_inc<SOFTMAX_REGS>();
   } else if (warp < 12) {
-    regs_dec<WIDEN_REGS>();
+    regs_dec<CORR_REGS>();
   } else {
     regs_dec<ISSUE_REGS>();
   }
@@ -259,27 +287,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
     const int X = warp >> 2, wq = warp & 3;
     if (X == 0 || hasB) {
       const uint32_t row = tid & 127;
-      uint8_t* qtile = sm + (X ? Smem::QB : Smem::QA);
       auto wait_all = [&](int b, uint32_t parity, uint32_t site) {
         return __all_sync(0xffffffffu, mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site));
       };
       bool ok = true;
       {
-        // widen this thread's packed Q row
-        const uint4* src = reinterpret_cast<const uint4*>(a.q4 + ((size_t)bh * P.N_pad + (size_t)(qt0 + X) * TILE + row) * (D / 2));
-        uint4 qp[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) qp[h] = __ldg(src + h);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint4 c0, c1;
-          widen16(qp[h], c0, c1);
-          *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h)) = c0;
-          *reinterpret_cast<uint4*>(qtile + sw128_off(row, 2 * h + 1)) = c1;
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_QFULL]);
         const int grow = (qt0 + X) * TILE + (int)row;
         const float kq = __fmul_rn(a.sq[(size_t)bh * nblk + grow / QK_BLOCK], LOG2E / (SQRT_D * 256.0f));
         const float* skb = a.sk + (size_t)bh * nblk;
@@ -332,6 +344,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const bool moved = j > 0 && m_new > m;
           const float alpha = moved ? ex2(m - m_new) : 1.0f;
           m = m_new;
+          // hand the O rescale of this row to the correction warp of the same
+          // TMEM lanes: acc * alpha = (2 acc * round(2^31 alpha)) >> 32
+          reinterpret_cast<int*>(sm + Smem::CQ)[X * 128 + row] =
+              moved ? __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f)) : NO_RESCALE;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_CREQ + X * 4 + wq]);
           const float negm = -m;
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
           // 64-key half whose largest x is below -5 holds only zero codes.
@@ -374,22 +392,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           }
           tmem_st32(tS + P_COL, pw);
           l = fmaf(l, alpha, (float)L);
-          // rows whose max moved: acc *= alpha before P.V(j) adds to it (the
-          // arrival of S(j) means P.V(j-1) has landed)
-          if (__any_sync(0xffffffffu, moved)) {
-            // acc * alpha = (2 acc * round(2^31 alpha)) >> 32, |acc| < 2^28
-            const int aq = __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f));
-            uint32_t acc[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
-            tmem_wait_ld();
-            if (moved) {
-#pragma unroll
-              for (int e = 0; e < 128; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
-          }
           if (dbg_tile && j == a.dbg_kv) {
 #pragma unroll
             for (int n = 0; n < 128; ++n) {
@@ -434,53 +436,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       }
     }
   } else if (warp < 12) {
-    // ------------------------------------------------------------ widen INT4 -> INT8
-    const int wt = tid - 256, rsub = wt >> 2, h = wt & 3;
-    for (int j = 0; j < nt; ++j) {
-      const int st = j % PK_STAGES, s = j % OP_STAGES;
-      bool ok = mbar_wait_abortable(&bar[B_PK_FULL + st], (j / PK_STAGES) & 1, abort_flag, limit, err, 0x4401);
-      if (ok && j >= OP_STAGES)
-        ok = mbar_wait_abortable(&bar[B_OP_EMPTY + s], ((j / OP_STAGES) - 1) & 1, abort_flag, limit, err, 0x4402);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      const uint8_t* src = sm + Smem::PK + st * 16384;
-      uint8_t* dst = sm + Smem::OP + s * 32768;
-#pragma unroll 4
-      for (int pass = 0; pass < 8; ++pass) {
-        const int r = pass * 32 + rsub;   // rows 0..127: K, 128..255: V^T
-        const uint4 u = *reinterpret_cast<const uint4*>(src + r * 64 + h * 16);
-        uint4 c0, c1;
-        widen16(u, c0, c1);
-        uint8_t* tile = dst + (r >> 7) * 16384;
-        *reinterpret_cast<uint4*>(tile + sw128_off(r & 127, 2 * h)) = c0;
-        *reinterpret_cast<uint4*>(tile + sw128_off(r & 127, 2 * h + 1)) = c1;
+    // ------------------------------------------------------------ O correction
+    // Per step j: rescale O_A and O_B for the rows whose max moved at tile j
+    // (after P.V(j-1), before P.V(j)).  Correction warp cw serves TMEM lanes
+    // 32 cw .. 32 cw + 31 of both query tiles.
+    const int cw = warp - 8;
+    auto correct = [&](int X, int j) -> bool {
+      // S_X(j) has landed, so P.V(j-1) has too; the softmax warp of these
+      // lanes has published its rows' factors for tile j
+      bool ok = mbar_wait_abortable(&bar[B_S_FULL + X], j & 1, abort_flag, limit, err, 0x4403);
+      if (ok) ok = mbar_wait_abortable(&bar[B_CREQ + X * 4 + cw], j & 1, abort_flag, limit, err, 0x4404);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc_fence_after();
+      const int aq = reinterpret_cast<const int*>(sm + Smem::CQ)[X * 128 + cw * 32 + lane];
+      if (__any_sync(0xffffffffu, aq != NO_RESCALE)) {
+        const uint32_t tO = tbase + 256 + X * 128 + ((uint32_t)(cw * 32) << 16);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t acc[32];
+          tmem_ld32(tO + 32 * c, acc);
+          tmem_wait_ld();
+          if (aq != NO_RESCALE) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
+          }
+          tmem_st32(tO + 32 * c, acc);
+        }
+        tmem_wait_st();
       }
-      fence_async_smem();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[B_OP_FULL + s]);
-        mbar_arrive(&bar[B_PK_EMPTY + st]);
-      }
+      if (lane == 0) mbar_arrive(&bar[B_P_FULL + X]);
+      return true;
+    };
+    bool ok = true;
+    for (int j = 0; ok && j < nt; ++j) {
+      ok = correct(0, j);
+      if (ok && hasB) ok = correct(1, j);
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ bulk-copy producer
+    // The INT8 operand images are laid out as the MMA reads them (128-byte
+    // swizzled, K-major), so every tile is one contiguous 16 KB copy.
     if (lane == 0) {
-      const uint8_t* kb = a.k4 + (size_t)bh * P.N_pad * (D / 2);
-      const uint8_t* vb = a.v4t + (size_t)bh * P.N_pad * (D / 2);
+      const uint8_t* qsrc = a.qimg + ((size_t)bh * nt + qt0) * 16384;
+      mbar_expect_tx(&bar[B_QFULL], hasB ? 32768u : 16384u);
+      bulk_g2s(sm + Smem::QA, qsrc, 16384, &bar[B_QFULL]);
+      if (hasB) bulk_g2s(sm + Smem::QB, qsrc + 16384, 16384, &bar[B_QFULL]);
+      const uint8_t* kb = a.kimg + (size_t)bh * nt * 16384;
+      const uint8_t* vb = a.vimg + (size_t)bh * nt * 16384;
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
-        const int st = j % PK_STAGES;
-        if (j >= PK_STAGES && !mbar_wait_abortable(&bar[B_PK_EMPTY + st], ((j / PK_STAGES) - 1) & 1, abort_flag,
+        const int st = j % OP_STAGES;
+        if (j >= OP_STAGES && !mbar_wait_abortable(&bar[B_OP_EMPTY + st], ((j / OP_STAGES) - 1) & 1, abort_flag,
                                                    limit, err, 0x4201))
           break;
-        uint8_t* dst = sm + Smem::PK + st * 16384;
-        mbar_expect_tx(&bar[B_PK_FULL + st], 16384u);
-        bulk_g2s(dst, kb + (size_t)j * 8192, 8192, &bar[B_PK_FULL + st]);
-        bulk_g2s(dst + 8192, vb + (size_t)j * 8192, 8192, &bar[B_PK_FULL + st]);
+        uint8_t* dst = sm + Smem::OP + st * 32768;
+        mbar_expect_tx(&bar[B_OP_FULL + st], 32768u);
+        bulk_g2s(dst, kb + (size_t)j * 16384, 16384, &bar[B_OP_FULL + st]);
+        bulk_g2s(dst + 16384, vb + (size_t)j * 16384, 16384, &bar[B_OP_FULL + st]);
         issued = j + 1;
       }
       if (*abort_flag) {   // let every copy still in flight land before the CTA exits
-        for (int j = issued > PK_STAGES ? issued - PK_STAGES : 0; j < issued; ++j)
-          mbar_wait(&bar[B_PK_FULL + j % PK_STAGES], (j / PK_STAGES) & 1, limit, err, 0x4204);
+        mbar_wait(&bar[B_QFULL], 0, limit, err, 0x4203);
+        for (int j = issued > OP_STAGES ? issued - OP_STAGES : 0; j < issued; ++j)
+          mbar_wait(&bar[B_OP_FULL + j % OP_STAGES], (j / OP_STAGES) & 1, limit, err, 0x4204);
       }
     }
   } else if (warp == 13 || warp == 14) {
@@ -552,7 +572,16 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
   e = cudaFuncGetAttributes(&fa, int4_attn_kernel);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-  KernelArgs a{p, q4, k4, v4t, sq, sk, sv, o, static_cast<WsHeader*>(ws), wait_limit(), dbg_bh, dbg_qtile, dbg_kv,
+  const WsLayout L = ws_layout(p);
+  uint8_t* img = static_cast<uint8_t*>(ws) + L.img;
+  const size_t plane = (size_t)p.BH * p.N_pad * D;   // bytes of one operand image set
+  const size_t units = plane / 32;                   // 16 packed bytes -> 32 image bytes
+  expand_kernel<<<dim3((unsigned)((units + 255) / 256), 3), 256, 0, st>>>(q4, k4, v4t, img, img + plane,
+                                                                          img + 2 * plane, units);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  KernelArgs a{p, img, img + plane, img + 2 * plane, sq, sk, sv, o, static_cast<WsHeader*>(ws), wait_limit(),
+               dbg_bh, dbg_qtile, dbg_kv,
                dbg_s, dbg_p};
   const int n_qt = p.N_pad / TILE;
   const dim3 grid = dbg_s ? dim3(1, 1) : dim3((n_qt + 1) / 2, p.BH);

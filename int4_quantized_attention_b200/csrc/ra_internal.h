@@ -37,7 +37,10 @@ struct WsHeader {
 struct WsLayout {
   size_t tables;                // float4 [n_tab]
   size_t vamax;                 // uint32 [BH][128]: fp32 bits of per-channel amax of V
-  size_t base_bytes;            // end of the part every call needs
+  size_t pro_bytes;             // end of the part the prologue needs
+  size_t img;                   // INT4 attention: INT8 operand images of Q, K, V^T,
+                                // 3 x [BH][N_pad / 128][16 KB]
+  size_t base_bytes;            // end of the part the INT4 path needs
   size_t qr, kr, vt;            // FP16 path: fp16 [BH][N_pad][128] x2, fp16 [BH][128][N_pad]
   size_t total_fp16;
 };
@@ -51,6 +54,9 @@ inline WsLayout ws_layout(const Prob& p) {
   o = align256(o + sizeof(float) * 4 * (size_t)p.n_tab);
   L.vamax = o;
   o = align256(o + sizeof(uint32_t) * (size_t)p.BH * D);
+  L.pro_bytes = o;
+  L.img = o;
+  o = align256(o + 3 * (size_t)p.BH * p.N_pad * D);
   L.base_bytes = o;
   size_t plane = (size_t)p.BH * p.N_pad * D * 2;
   L.qr = o;

@@ -61,11 +61,11 @@ extern "C" ra_status ra_rotate_quantize_qkv_noalloc(const ra_problem* p, const v
     return RA_ERR_INVALID_ARG;
   }
   const ra::WsLayout L = ra::ws_layout(P);
-  if (L.base_bytes > RA_NOALLOC_SCRATCH_BYTES) {
+  if (L.pro_bytes > RA_NOALLOC_SCRATCH_BYTES) {
     char msg[200];
     snprintf(msg, sizeof(msg),
              "problem needs %zu bytes of scratch; the fixed scratch holds %u (RA_NOALLOC_SCRATCH_BYTES)",
-             L.base_bytes, (unsigned)RA_NOALLOC_SCRATCH_BYTES);
+             L.pro_bytes, (unsigned)RA_NOALLOC_SCRATCH_BYTES);
     ra::set_error_detail(msg);
     return RA_ERR_WORKSPACE;
   }

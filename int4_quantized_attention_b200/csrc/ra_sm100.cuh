@@ -139,6 +139,26 @@ __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t pari
   }
 }
 
+// Waits as mbar_wait_abortable, but polls without suspending the thread: the
+// lowest wake-up latency, for waits on the critical path of a pipeline (each
+// poll costs an issue slot, so keep it to one thread or warp per SM quarter).
+__device__ __forceinline__ bool mbar_spin_abortable(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                    uint64_t limit_ns, DeviceErr* err, uint32_t site) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        report(err, DEVERR_TIMEOUT, site);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- bulk copy
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes must be
 // a multiple of 16, both addresses 16-byte aligned).
