@@ -7,33 +7,32 @@
 // (Sec. 4.2 as summarised by the referee report; free-parameter ledger) --
 // with the zero-point corrected through the V column sums.
 //
-// One CTA = one (batch*head, pair of 128-row query tiles A and B); 512
-// threads in four warpgroups:
+// One CTA = one (batch*head, pair of 128-row query tiles A and B); 384
+// threads in three warpgroups:
 //   WG0 (warps 0-3)    softmax of tile A, thread t = query row t = TMEM lane t
 //   WG1 (warps 4-7)    softmax of tile B
-//   WG2 (warps 8-11)   O correction: rescales the accumulator rows whose max
-//                      moved, for both tiles, off the softmax warps' path
-//   WG3 warp 12        bulk-copy producer: the two Q operand tiles once, then
+//   WG2 warp 8         bulk-copy producer: the two Q operand tiles once, then
 //                      the K and V^T operand tiles (16 KB each) into a
-//                      5-stage ring
-//       warps 13, 14   MMA issuers, one thread per query tile (warp 13 also
+//                      3-stage ring
+//       warps 9, 10    MMA issuers, one thread per query tile (warp 9 also
 //                      owns the TMEM allocation)
-//       warp 15        writes the constant bf16 operand at start-up
+//       warp 11        writes the constant bf16 operand at start-up
 // The packed INT4 inputs are expanded once per call, by expand_kernel, into
 // INT8 operand images laid out exactly as the MMAs read them from SMEM, so
 // the attention kernel itself only copies tiles.
+//
 // TMEM (512 columns): S_A | S_B | O_A | O_B, 128 int32 columns each.  The P
-// operand of a tile (128 rows x 128 u8 = 32 columns) is stored by the softmax
-// threads into the last 32 columns of their own S region once S is in
-// registers, and read from there by the P.V MMA (A operand in TMEM).
-// MMA order per query tile X: S_X(0); then for every tile j: O_X += W_X(j)
-// V(j), S_X(j+1).  Each tile has its own issuing thread, blocked on that
-// tile's barriers, so the tensor core runs one tile's MMAs while the other
-// tile's softmax runs (ping-pong) with no polling between them.  Because the
-// MMAs of one thread complete in issue order, the arrival of S_X(j+1) also
-// means that P.V(j) has landed: O_X may be rescaled right then, and must be
-// before P.V(j+1), whose issue waits for the correction warps as well as for
-// the softmax warps.
+// operand (128 rows x 128 u8 = 16 KB) goes to SMEM, double-buffered per
+// query tile, laid out like a Q tile.  So the S columns are free as soon as
+// the softmax warps hold S in registers: tile X's thread issues S_X(j+1)
+// right then, and S_X(j+1) is ready when the softmax finishes tile j; it
+// issues O_X += W_X(j) V(j) once the four softmax warps have stored W_X(j).
+// The two tiles' threads share the tensor core and the operand ring, which
+// is refilled once both have consumed a stage.
+//
+// A row whose running max moves has its int32 accumulator rescaled in TMEM by
+// its own softmax thread, after P.V(j-1) has landed (issued a whole tile
+// earlier) and before it releases W(j).
 //
 // S_X(j) starts as 1.5 * 2^23 in every accumulator (one bf16 MMA with a
 // constant operand), so after the integer MMAs add 256 S the accumulator bits
@@ -43,10 +42,9 @@
 // The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15], fed as an
 // unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
 // sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
-// The int32 P.V accumulator stays in TMEM across tiles; a row whose running
-// max moves has its accumulator rescaled in place with an integer multiply by
-// round(2^31 * exp(m_old - m_new)) (exp(...) is exactly 1 for every other
-// row).  The normaliser l is the running sum of w.
+// The int32 P.V accumulator stays in TMEM across tiles; the rescale is an
+// integer multiply by round(2^31 * exp(m_old - m_new)) (exp(...) is exactly
+// 1 for every other row).  The normaliser l is the running sum of w.
 //
 // INT4 codes are expanded to 16*code (the nibble placed in the high half of
 // the byte), so S comes out as 256*S and P.V as 16*P.V, exactly; both factors
@@ -65,15 +63,13 @@
 namespace ra {
 namespace {
 
-constexpr int NUM_THREADS = 512;
-constexpr int OP_STAGES = 5;   // INT8 K / V^T operand tiles (bulk copies)
-// Register split: launched at LAUNCH_REGS per thread (512 x 128 = 65536); the
-// correction warpgroup drops to CORR_REGS, the copy/MMA warpgroup to
-// ISSUE_REGS, the two softmax warpgroups rise to SOFTMAX_REGS:
-// 256 x 192 + 128 x 64 + 128 x 64 = 65536.
-constexpr int LAUNCH_REGS = 128, SOFTMAX_REGS = 192, CORR_REGS = 64, ISSUE_REGS = 64;
-static_assert(256 * SOFTMAX_REGS + 128 * CORR_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS,
-              "register split");
+constexpr int NUM_THREADS = 384;
+constexpr int OP_STAGES = 3;   // INT8 K / V^T operand tiles (bulk copies)
+// Register split: launched at LAUNCH_REGS per thread (384 x 168 = 64512);
+// the copy/MMA warpgroup drops to ISSUE_REGS, the two softmax warpgroups
+// rise to SOFTMAX_REGS: 256 x 208 + 128 x 88 = 64512.
+constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 208, ISSUE_REGS = 88;
+static_assert(256 * SOFTMAX_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 
 constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
 constexpr uint32_t IDESC_PV = make_idesc(2, 0, 1, 128, 128);   // s32 += u8 x s8
@@ -83,22 +79,22 @@ constexpr float SQRT_D = 11.313708498984761f;
 constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
 constexpr int MAGIC_BITS = 0x4B400000;
 constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6), still exact through MAGIC
-constexpr uint32_t P_COL = 96;    // P operand: columns 96..127 of the tile's S region
 
 struct Smem {
   static constexpr uint32_t QA = 0, QB = 16384;   // INT8 Q operand tiles
-  static constexpr uint32_t OP = 32768;           // 5 x 32 KB: INT8 K (+0), V^T (+16 KB)
+  static constexpr uint32_t OP = 32768;           // 3 x 32 KB: INT8 K (+0), V^T (+16 KB)
+  static constexpr uint32_t P = 131072;           // [tile][j % 2] 16 KB u8 P operands, laid out like Q
   static constexpr uint32_t CT = 196608;          // 4 KB: bf16 operand that sets S to 1.5 * 2^23
-  static constexpr uint32_t CQ = 200704;          // 2 x 128 ints: per-row O rescale factors
-  static constexpr uint32_t BAR = 201728;
+  static constexpr uint32_t BAR = 200704;
   static constexpr uint32_t BYTES = BAR + 512;
 };
 
+// P_FULL[tile][b] and PV_DONE[tile][b] serve the KV tiles j with j % 2 == b:
+// a softmax warp may store P(j+1) while another still works on P(j).
 enum : int {
-  B_OP_FULL = 0, B_OP_EMPTY = 5, B_QFULL = 10, B_S_FULL = 11, B_P_FULL = 13, B_O_DONE = 15, B_DRAIN = 17,
-  B_CREQ = 19, NBAR = 27
+  B_OP_FULL = 0, B_OP_EMPTY = 3, B_QFULL = 6, B_S_FULL = 7, B_S_EMPTY = 9, B_P_FULL = 11, B_PV_DONE = 15,
+  B_DRAIN = 19, NBAR = 21
 };
-constexpr int NO_RESCALE = -1;   // rescale factor of a row whose max stayed
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -140,17 +136,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
       "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]^T for kind::i8: A holds 4 bytes of a row per
-// 32-bit column, row m in lane m.
-__device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                               uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -246,20 +231,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar[B_S_FULL + i], 1);
-      mbar_init(&bar[B_P_FULL + i], 8);   // 4 softmax warps + 4 correction warps
-      mbar_init(&bar[B_O_DONE + i], 1);
+      mbar_init(&bar[B_S_EMPTY + i], 4);  // the softmax warps have S in registers
+      mbar_init(&bar[B_P_FULL + 2 * i], 4);
+      mbar_init(&bar[B_P_FULL + 2 * i + 1], 4);
+      mbar_init(&bar[B_PV_DONE + 2 * i], 1);
+      mbar_init(&bar[B_PV_DONE + 2 * i + 1], 1);
       mbar_init(&bar[B_DRAIN + i], 1);
     }
     mbar_init(&bar[B_QFULL], 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&bar[B_CREQ + i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == 9) {
     tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
-  if (warp == 15) {
+  if (warp == 11) {
     // bf16 2048 in columns 0..2 of every row, zero elsewhere: used as both
     // operands, A B^T = 3 * 2048^2 = 1.5 * 2^23 in every accumulator, whose
     // bits 0x4B400000 the integer S MMAs then add 256 S to
@@ -276,8 +263,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   const uint32_t tbase = *tslot;
   if (warp < 8) {
     regs_inc<SOFTMAX_REGS>();
-  } else if (warp < 12) {
-    regs_dec<CORR_REGS>();
   } else {
     regs_dec<ISSUE_REGS>();
   }
@@ -307,13 +292,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
             skn0 = __ldg(skb + 2 * j + 2);
             skn1 = __ldg(skb + 2 * j + 3);
           }
-          // S_X(j) has landed -- and with it every earlier MMA, P.V(j-1) included
           if (!(ok = wait_all(B_S_FULL + X, j & 1, 0x4102))) break;
           tc_fence_after();
           uint32_t s[128];
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
           tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_S_EMPTY + X]);   // S_X(j+1) may overwrite the S columns
           const int nvalid = (j == nt - 1) ? tail : TILE;
           if (dbg_tile && j == a.dbg_kv) {   // S = (256 S) >> 8, exactly
 #pragma unroll
@@ -344,12 +331,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const bool moved = j > 0 && m_new > m;
           const float alpha = moved ? ex2(m - m_new) : 1.0f;
           m = m_new;
-          // hand the O rescale of this row to the correction warp of the same
-          // TMEM lanes: acc * alpha = (2 acc * round(2^31 alpha)) >> 32
-          reinterpret_cast<int*>(sm + Smem::CQ)[X * 128 + row] =
-              moved ? __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f)) : NO_RESCALE;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[B_CREQ + X * 4 + wq]);
           const float negm = -m;
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
           // 64-key half whose largest x is below -5 holds only zero codes.
@@ -390,7 +371,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               pw[k] &= keep;
             }
           }
-          tmem_st32(tS + P_COL, pw);
+          // rows whose max moved: acc *= alpha after P.V(j-1) has landed (it
+          // was issued a whole tile ago) and before P.V(j) adds to it
+          if (__any_sync(0xffffffffu, moved)) {
+            if (!(ok = wait_all(B_PV_DONE + 2 * X + ((j - 1) & 1), ((j - 1) >> 1) & 1, 0x4104))) break;
+            tc_fence_after();
+            // acc * alpha = (2 acc * round(2^31 alpha)) >> 32, |acc| < 2^28
+            const int aq = __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f));
+            uint32_t acc[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
+            tmem_wait_ld();
+            if (moved) {
+#pragma unroll
+              for (int e = 0; e < 128; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
+            tmem_wait_st();
+          }
+          // P buffer j % 2 is free again once P.V(j-2) has read it
+          if (j >= 2 && !(ok = wait_all(B_PV_DONE + 2 * X + (j & 1), ((j - 2) >> 1) & 1, 0x4103))) break;
+          {
+            uint8_t* prow = sm + Smem::P + (2 * X + (j & 1)) * 16384;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(prow + sw128_off(row, c)) =
+                  make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            fence_async_smem();
+          }
           l = fmaf(l, alpha, (float)L);
           if (dbg_tile && j == a.dbg_kv) {
 #pragma unroll
@@ -399,12 +408,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               a.dbg_p[row * TILE + n] = n < nvalid ? (int8_t)(w - 8) : (int8_t)-128;
             }
           }
-          tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[B_P_FULL + X]);
+          if (lane == 0) mbar_arrive(&bar[B_P_FULL + 2 * X + (j & 1)]);
         }
-        if (ok) ok = wait_all(B_O_DONE + X, 0, 0x4105);
+        // the last P.V has landed
+        if (ok) ok = wait_all(B_PV_DONE + 2 * X + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, 0x4105);
         if (ok) {
           // epilogue: O = acc * s_V / (16 l) -> fp16; loads are warp-collective,
           // stores only for rows < N
@@ -435,46 +444,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         }
       }
     }
-  } else if (warp < 12) {
-    // ------------------------------------------------------------ O correction
-    // Per step j: rescale O_A and O_B for the rows whose max moved at tile j
-    // (after P.V(j-1), before P.V(j)).  Correction warp cw serves TMEM lanes
-    // 32 cw .. 32 cw + 31 of both query tiles.
-    const int cw = warp - 8;
-    auto correct = [&](int X, int j) -> bool {
-      // S_X(j) has landed, so P.V(j-1) has too; the softmax warp of these
-      // lanes has published its rows' factors for tile j
-      bool ok = mbar_wait_abortable(&bar[B_S_FULL + X], j & 1, abort_flag, limit, err, 0x4403);
-      if (ok) ok = mbar_wait_abortable(&bar[B_CREQ + X * 4 + cw], j & 1, abort_flag, limit, err, 0x4404);
-      if (!__all_sync(0xffffffffu, ok)) return false;
-      tc_fence_after();
-      const int aq = reinterpret_cast<const int*>(sm + Smem::CQ)[X * 128 + cw * 32 + lane];
-      if (__any_sync(0xffffffffu, aq != NO_RESCALE)) {
-        const uint32_t tO = tbase + 256 + X * 128 + ((uint32_t)(cw * 32) << 16);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t acc[32];
-          tmem_ld32(tO + 32 * c, acc);
-          tmem_wait_ld();
-          if (aq != NO_RESCALE) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
-          }
-          tmem_st32(tO + 32 * c, acc);
-        }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[B_P_FULL + X]);
-      return true;
-    };
-    bool ok = true;
-    for (int j = 0; ok && j < nt; ++j) {
-      ok = correct(0, j);
-      if (ok && hasB) ok = correct(1, j);
-    }
-  } else if (warp == 12) {
+  } else if (warp == 8) {
     // ------------------------------------------------------------ bulk-copy producer
     // The INT8 operand images are laid out as the MMA reads them (128-byte
     // swizzled, K-major), so every tile is one contiguous 16 KB copy.
@@ -503,45 +473,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           mbar_wait(&bar[B_OP_FULL + j % OP_STAGES], (j / OP_STAGES) & 1, limit, err, 0x4204);
       }
     }
-  } else if (warp == 13 || warp == 14) {
+  } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers
-    // One thread per query tile, each blocked on its own tile's barriers, so
-    // each tile's MMAs go out as soon as its P operand is stored.  Tile X's
-    // step j is O_X += W_X(j-1) V(j-1), then S_X(j) = Q_X K(j)^T (operand
-    // stage j).  MMAs of one thread complete in issue order; the two threads'
-    // MMAs touch disjoint TMEM and only read the shared operand stages, whose
-    // release counts one commit from each thread.
-    const int X = warp - 13;
+    // One thread per query tile, each blocked on its own tile's barriers.
+    // Tile X computes S_X(j+1) = Q_X K(j+1)^T as soon as its softmax warps
+    // have S_X(j) in registers, so the next S is ready when they finish tile
+    // j; O_X += W_X(j) V(j) follows once W_X(j) is stored (and O_X rescaled).
+    // MMAs of one thread complete in issue order; the two threads' MMAs touch
+    // disjoint TMEM and only read the shared operand stages, whose release
+    // counts one commit from each thread.
+    const int X = warp - 9;
     if (lane == 0 && (X == 0 || hasB)) {
       const uint32_t qa = smem_u32(sm + (X ? Smem::QB : Smem::QA));
+      const uint32_t pbase = smem_u32(sm + Smem::P + 2 * X * 16384);
       const uint32_t op = smem_u32(sm + Smem::OP);
       const uint64_t dc = plain_desc(smem_u32(sm + Smem::CT));
       const uint32_t tS = tbase + X * 128, tO = tbase + 256 + X * 128;
       auto wait = [&](int b, uint32_t parity, uint32_t site) {
         return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
       };
-      bool ok = wait(B_QFULL, 0, 0x4301);
-      for (int j = 0; ok && j <= nt; ++j) {
-        if (j > 0 && !(ok = wait(B_P_FULL + X, (j - 1) & 1, 0x4302))) break;
-        if (j < nt && !(ok = wait(B_OP_FULL + j % OP_STAGES, (j / OP_STAGES) & 1, 0x4303))) break;
+      auto issue_S = [&](int j) {   // S_X(j): set to 1.5 * 2^23, then += 256 Q_X K(j)^T
+        const uint32_t kt = op + (j % OP_STAGES) * 32768;
+        umma_f16(tS, dc, dc, IDESC_INIT, 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, 1);
+        umma_commit(&bar[B_S_FULL + X]);
+      };
+      bool ok = wait(B_QFULL, 0, 0x4301) && wait(B_OP_FULL, 0, 0x4302);
+      if (ok) {
         tc_fence_after();
-        if (j > 0) {   // O_X += W_X(j-1) V(j-1), W from TMEM
-          const uint32_t vt = op + ((j - 1) % OP_STAGES) * 32768 + 16384;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_i8_tmem_a(tO, tS + P_COL + 8 * kk, sw128_desc(vt + 32 * kk), IDESC_PV, (j > 1) || (kk > 0));
-          umma_commit(&bar[B_OP_EMPTY + (j - 1) % OP_STAGES]);
+        issue_S(0);
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 1 < nt) {
+          if (!(ok = wait(B_S_EMPTY + X, j & 1, 0x4303))) break;
+          if (!(ok = wait(B_OP_FULL + (j + 1) % OP_STAGES, ((j + 1) / OP_STAGES) & 1, 0x4304))) break;
+          tc_fence_after();
+          issue_S(j + 1);
         }
-        if (j < nt) {   // S_X(j): set to 1.5 * 2^23, then += 256 Q_X K(j)^T
-          const uint32_t kt = op + (j % OP_STAGES) * 32768;
-          umma_f16(tS, dc, dc, IDESC_INIT, 0);
+        if (!(ok = wait(B_P_FULL + 2 * X + (j & 1), (j >> 1) & 1, 0x4305))) break;
+        tc_fence_after();
+        const uint32_t vt = op + (j % OP_STAGES) * 32768 + 16384;   // O_X += W_X(j) V(j)
+        const uint32_t pa = pbase + (j & 1) * 16384;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, 1);
-          umma_commit(&bar[B_S_FULL + X]);
-        } else {
-          umma_commit(&bar[B_O_DONE + X]);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          umma_i8(tO, sw128_desc(pa + 32 * kk), sw128_desc(vt + 32 * kk), IDESC_PV, (j > 0) || (kk > 0));
+        umma_commit(&bar[B_PV_DONE + 2 * X + (j & 1)]);
+        umma_commit(&bar[B_OP_EMPTY + j % OP_STAGES]);
       }
       // every MMA this thread issued completes before TMEM is released
       umma_commit(&bar[B_DRAIN + X]);
@@ -551,7 +530,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
