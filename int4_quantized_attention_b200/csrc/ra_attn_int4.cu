@@ -207,6 +207,10 @@ struct KernelArgs {
   int8_t* dbg_p;
 };
 
+// DBG: the test-only instance that runs one CTA at the given tiles and
+// exports one S tile and its P codes; the production instance carries none
+// of that code.
+template <bool DBG>
 __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
@@ -216,7 +220,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Prob& P = a.P;
-  const bool dbg_run = a.dbg_s != nullptr;
+  constexpr bool dbg_run = DBG;
   const int n_qt = P.N_pad / TILE, nt = n_qt, nblk = P.N_pad / QK_BLOCK;
   const int qt0 = 2 * (blockIdx.x + (dbg_run ? a.dbg_qt / 2 : 0));
   const int bh = blockIdx.y + (dbg_run ? a.dbg_bh : 0);
@@ -542,13 +546,14 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
                                   const float* sq, const float* sk, const float* sv, __half* o, void* ws, int dbg_bh,
                                   int dbg_qtile, int dbg_kv, int32_t* dbg_s, int8_t* dbg_p, cudaStream_t st) {
   const int smem = Smem::BYTES + 1024;   // > half the SM: one CTA per SM owns all 512 TMEM columns
-  cudaError_t e = cudaFuncSetAttribute(int4_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kernel = dbg_s ? int4_attn_kernel<true> : int4_attn_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   // The setmaxnreg split assumes the kernel launches with LAUNCH_REGS per
   // thread; with fewer, the softmax warpgroups' increase could never be
   // granted.  Refuse to launch rather than risk that.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, int4_attn_kernel);
+  e = cudaFuncGetAttributes(&fa, kernel);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
   const WsLayout L = ws_layout(p);
@@ -564,7 +569,7 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
                dbg_s, dbg_p};
   const int n_qt = p.N_pad / TILE;
   const dim3 grid = dbg_s ? dim3(1, 1) : dim3((n_qt + 1) / 2, p.BH);
-  int4_attn_kernel<<<grid, NUM_THREADS, smem, st>>>(a);
+  kernel<<<grid, NUM_THREADS, smem, st>>>(a);
   return cudaGetLastError();
 }
 
