@@ -4,13 +4,29 @@
 // RotateAttention (arXiv 2607.02584) review page: accuracy-sensitive
 // attention calls (first/last denoising steps and DiT blocks) stay in FP16
 // (abstract, Sec. 5.1); this is that path: FlashAttention over the RoPE-encoded
-// fp16 Q and K with fp32 accumulation in tensor memory.
+// fp16 Q and K, P in fp16, fp32 accumulation in tensor memory.
 //
-// One CTA per (batch*head, 128-row query tile); thread t = query row t = TMEM
-// lane t.  Per 128-key tile: operands copied into 128-byte-swizzled K-major
-// SMEM (fp16 rows are 256 bytes: two swizzle atoms), S = Q K^T on
-// tcgen05.mma.kind::f16 into TMEM, online softmax in registers, P in fp16 to
-// SMEM, O += P V into TMEM; rows whose max moved rescale O in place.
+// One CTA = one (batch*head, pair of 128-row query tiles A and B); 384
+// threads:
+//   warps 0-3 / 4-7   softmax of tile A / B; thread t = query row t = TMEM lane t
+//   warp 8            bulk copies: the two Q tiles once, then the K tiles
+//   warp 11           bulk copies of the V^T tiles
+//   warps 9, 10       MMA issuers, one thread per query tile (warp 9 owns TMEM)
+// The FP16 prologue writes Q, K and V^T as operand images: per 128-row tile,
+// two 16 KB 128-byte-swizzled K-major atoms (elements 0..63 and 64..127 of
+// every row), so each tile is one 32 KB bulk copy.  K and V^T have separate
+// 2-stage rings: a K stage is free once both tiles' S MMAs have read it, a V
+// stage once both tiles' P.V MMAs have.
+// TMEM: S_A | S_B | O_A | O_B, 128 fp32 columns each.  The softmax threads
+// load S_X(j), then store P_X(j) as fp16 pairs into the upper 64 columns of
+// S_X, from where the P.V MMAs read their A operand.  Tile X's thread issues,
+// per KV tile j: O_X += P_X(j) V(j) (once P_X(j) is stored), then S_X(j+1)
+// (which overwrites the P columns, so it follows the P.V in issue order).
+// MMAs of one thread complete in issue order: S_X(j+1) landing means P.V(j)
+// has too, so the softmax may rescale O_X (fp32) right then.
+// A 64-key half whose largest exponent is below -26 holds only P values that
+// round to zero in fp16; its exponentials are skipped when that is so for
+// every row of a warp (the fp16 operand is the same).
 #include <cuda_fp16.h>
 #include <cstdint>
 
@@ -19,179 +35,278 @@
 namespace ra {
 namespace {
 
-constexpr uint32_t IDESC_F16 = make_idesc(1, 0, 0, 128, 128);   // f32 += f16 x f16
+namespace f16 {
+constexpr int NUM_THREADS = 384;
+constexpr int STAGES = 2;
+constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 208, ISSUE_REGS = 88;
+static_assert(256 * SOFTMAX_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
+constexpr uint32_t IDESC = make_idesc(1, 0, 0, 128, 128);   // f32 += f16 x f16
 constexpr float LOG2E = 1.4426950408889634f;
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-// ---------------------------------------------------------------------------
-// FP16 attention (inputs position-encoded and V transposed by the FP16
-// prologue).  fp16 operands: a 128-element row is 256 bytes, i.e. two
-// 128-byte swizzle atoms ("K blocks") of 64 elements, 16 KB apart.
-struct F16Smem {
-  static constexpr uint32_t Q = 0, K = 32768, V = 65536, P = 98304, BAR = 131072, BYTES = BAR + 64;
+constexpr float SKIP_BELOW = -26.0f;                        // 2^-26 rounds to fp16 zero
+struct Smem {
+  static constexpr uint32_t QA = 0, QB = 32768;            // 32 KB Q tiles
+  static constexpr uint32_t K = 65536;                       // 2 x 32 KB
+  static constexpr uint32_t V = 131072;                      // 2 x 32 KB
+  static constexpr uint32_t BAR = 196608;
+  static constexpr uint32_t BYTES = BAR + 512;
 };
-
-__device__ __forceinline__ uint32_t f16_off(uint32_t row, uint32_t col) {   // element offset (bytes)
-  return (col >> 6) * 16384u + sw128_off(row, (col & 63) >> 3) + (col & 7) * 2;
-}
-
-// Copy one 256-byte fp16 row from global into the two-atom swizzled layout.
-__device__ __forceinline__ void copy_row_f16(uint8_t* tile, uint32_t row, const __half* __restrict__ src) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) *reinterpret_cast<uint4*>(tile + f16_off(row, 8 * c)) = __ldg(s + c);
-}
-
-__device__ __forceinline__ uint64_t f16_desc(uint32_t base, int kk) {   // K step kk of 16 elements
+enum : int {
+  B_KFULL = 0, B_KEMPTY = 2, B_VFULL = 4, B_VEMPTY = 6, B_QFULL = 8, B_SFULL = 9, B_PFULL = 11, B_ODONE = 13,
+  B_DRAIN = 15, NBAR = 17
+};
+// K step kk (16 elements) of a two-atom operand tile
+__device__ __forceinline__ uint64_t desc(uint32_t base, int kk) {
   return sw128_desc(base + (kk >> 2) * 16384u + (kk & 3) * 32u);
 }
+}  // namespace f16
 
-__global__ void __launch_bounds__(128, 1)
-    fp16_attn_kernel(Prob Pb, const __half* __restrict__ qr, const __half* __restrict__ kr,
-                     const __half* __restrict__ vt, __half* __restrict__ o, WsHeader* __restrict__ hdr,
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(f16::NUM_THREADS, 1)
+    fp16_attn_kernel(Prob Pb, const uint8_t* __restrict__ qimg, const uint8_t* __restrict__ kimg,
+                     const uint8_t* __restrict__ vimg, __half* __restrict__ o, WsHeader* __restrict__ hdr,
                      uint64_t limit) {
+  using namespace f16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
-  uint8_t* Qs = sm + F16Smem::Q;
-  uint8_t* Ks = sm + F16Smem::K;
-  uint8_t* Vs = sm + F16Smem::V;
-  uint8_t* Ps = sm + F16Smem::P;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + F16Smem::BAR);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + F16Smem::BAR + 32);
-  int* abort_flag = reinterpret_cast<int*>(sm + F16Smem::BAR + 40);
-
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int qt = blockIdx.x, bh = blockIdx.y;
-  const int N = Pb.N, N_pad = Pb.N_pad;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Smem::BAR);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Smem::BAR + 8 * NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Smem::BAR + 8 * NBAR + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = Pb.N_pad / TILE;
+  const int qt0 = 2 * blockIdx.x, bh = blockIdx.y;
+  const bool hasB = qt0 + 1 < nt;
   DeviceErr* err = &hdr->err;
+
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    mbar_init(&bar[2], 1);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&bar[B_KFULL + i], 1);
+      mbar_init(&bar[B_KEMPTY + i], hasB ? 2 : 1);
+      mbar_init(&bar[B_VFULL + i], 1);
+      mbar_init(&bar[B_VEMPTY + i], hasB ? 2 : 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar[B_SFULL + i], 1);
+      mbar_init(&bar[B_PFULL + i], 4);
+      mbar_init(&bar[B_ODONE + i], 1);
+      mbar_init(&bar[B_DRAIN + i], 1);
+    }
+    mbar_init(&bar[B_QFULL], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tslot, 256);
+  if (warp == 9) {
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
-  const int row = qt * TILE + tid;
-  copy_row_f16(Qs, tid, qr + ((size_t)bh * N_pad + row) * D);
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const uint32_t tS = tbase, tO = tbase + 128;
-  const uint32_t lane = (uint32_t)(warp * 32) << 16;
-  const uint32_t qs_addr = smem_u32(Qs), ks_addr = smem_u32(Ks), vs_addr = smem_u32(Vs), ps_addr = smem_u32(Ps);
-  const float cs = LOG2E / 11.313708498984761f;   // log2(e) / sqrt(128)
-  float m = -INFINITY, l = 0.0f;
-  const int ntiles = N_pad / TILE;
-  for (int j = 0; j < ntiles; ++j) {
-    copy_row_f16(Ks, tid, kr + ((size_t)bh * N_pad + (size_t)j * TILE + tid) * D);
-    copy_row_f16(Vs, tid, vt + ((size_t)bh * D + tid) * N_pad + (size_t)j * TILE);
-    fence_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) umma_f16(tS, f16_desc(qs_addr, kk), f16_desc(ks_addr, kk), IDESC_F16, kk > 0);
-      umma_commit(&bar[0]);
-    }
-    if (!mbar_wait(&bar[0], j & 1, limit, err, 0x2001)) *abort_flag = 1;
-    if (__syncthreads_or(*abort_flag)) break;
-    tc_fence_after();
-    uint32_t s[128];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) tmem_ld16(tS + lane + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&s[16 * c]));
-    tmem_wait_ld();
-    const int nvalid = min(TILE, N - j * TILE);
-    float tmax = -INFINITY;
-#pragma unroll
-    for (int n = 0; n < 128; ++n)
-      if (n < nvalid) tmax = fmaxf(tmax, __uint_as_float(s[n]));
-    tmax *= cs;
-    const float m_new = fmaxf(m, tmax);
-    const bool moved = (j > 0) && (m_new > m);
-    const float alpha = moved ? ex2(m - m_new) : 1.0f;
-    if (__any_sync(0xffffffffu, moved)) {
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t acc[16];
-        tmem_ld16(tO + lane + 16 * c, acc);
-        tmem_wait_ld();
-        if (moved) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) acc[e] = __float_as_uint(__uint_as_float(acc[e]) * alpha);
-        }
-        tmem_st16(tO + lane + 16 * c, acc);
-      }
-      tmem_wait_st();
-    }
-    m = m_new;
-    const float negm = -m;
-    float Lsum = 0.0f;
-#pragma unroll
-    for (int ch = 0; ch < 16; ++ch) {   // 8 keys per 16-byte chunk
-      uint32_t hv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int n = 8 * ch + 2 * e;
-        const float p0 = n < nvalid ? ex2(fmaf(__uint_as_float(s[n]), cs, negm)) : 0.0f;
-        const float p1 = n + 1 < nvalid ? ex2(fmaf(__uint_as_float(s[n + 1]), cs, negm)) : 0.0f;
-        Lsum += p0 + p1;
-        const __half2 h2 = __floats2half2_rn(p0, p1);
-        hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
-      *reinterpret_cast<uint4*>(Ps + f16_off(tid, 8 * ch)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    l = fmaf(l, alpha, Lsum);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        umma_f16(tO, f16_desc(ps_addr, kk), f16_desc(vs_addr, kk), IDESC_F16, (j > 0) || (kk > 0));
-      umma_commit(&bar[1]);
-    }
-    if (!mbar_wait(&bar[1], j & 1, limit, err, 0x2002)) *abort_flag = 1;
-    if (__syncthreads_or(*abort_flag)) break;
-    tc_fence_after();
+  if (warp < 8) {
+    regs_inc<SOFTMAX_REGS>();
+  } else {
+    regs_dec<ISSUE_REGS>();
   }
-  if (!*abort_flag) {
-    const float inv = 1.0f / l;
-#pragma unroll 1
-    for (int c = 0; c < 8; ++c) {
-      uint32_t acc[16];
-      tmem_ld16(tO + lane + 16 * c, acc);
-      tmem_wait_ld();
-      if (row < N) {
-        uint32_t hv[8];
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    const int X = warp >> 2, wq = warp & 3;
+    if (X == 0 || hasB) {
+      auto wait_all = [&](int b, uint32_t parity, uint32_t site) {
+        return __all_sync(0xffffffffu, mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site));
+      };
+      const int row = qt0 * TILE + X * TILE + (tid & 127);
+      const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+      const uint32_t tS = tbase + X * 128 + lane_off, tO = tbase + 256 + X * 128 + lane_off;
+      const float cs = LOG2E / 11.313708498984761f;   // log2(e) / sqrt(128)
+      const int tail = Pb.N - (nt - 1) * TILE;        // valid keys in the last tile, 1..128
+      float m = -INFINITY, l = 0.0f;
+      bool ok = true;
+      for (int j = 0; j < nt; ++j) {
+        // S_X(j) has landed -- and with it P.V(j-1)
+        if (!(ok = wait_all(B_SFULL + X, j & 1, 0x2101))) break;
+        tc_fence_after();
+        uint32_t s[128];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const __half2 h2 = __floats2half2_rn(__uint_as_float(acc[2 * e]) * inv, __uint_as_float(acc[2 * e + 1]) * inv);
-          hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+        tmem_wait_ld();
+        const int nvalid = (j == nt - 1) ? tail : TILE;
+        if (nvalid < TILE) {
+#pragma unroll
+          for (int n = 0; n < 128; ++n)
+            if (n >= nvalid) s[n] = 0xFF800000u;   // -inf: out of the max and the sum
         }
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * N + row) * D + 16 * c);
-        dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+        float mh[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          mh[c] = fmax3(__uint_as_float(s[16 * c]), __uint_as_float(s[16 * c + 1]), __uint_as_float(s[16 * c + 2]));
+#pragma unroll
+          for (int n = 3; n < 15; n += 2)
+            mh[c] = fmax3(mh[c], __uint_as_float(s[16 * c + n]), __uint_as_float(s[16 * c + n + 1]));
+          mh[c] = fmaxf(mh[c], __uint_as_float(s[16 * c + 15]));
+        }
+        const float mx0 = fmaxf(fmax3(mh[0], mh[1], mh[2]), mh[3]) * cs;
+        const float mx1 = fmaxf(fmax3(mh[4], mh[5], mh[6]), mh[7]) * cs;
+        const float m_new = fmaxf(m, fmaxf(mx0, mx1));
+        const bool moved = j > 0 && m_new > m;
+        const float alpha = moved ? ex2(m - m_new) : 1.0f;
+        m = m_new;
+        const float negm = -m;
+        // rows whose max moved: O *= alpha (P.V(j-1) has landed, P.V(j) not issued)
+        if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t acc[32];
+            tmem_ld32(tO + 32 * c, acc);
+            tmem_wait_ld();
+            if (moved) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = __float_as_uint(__uint_as_float(acc[e]) * alpha);
+            }
+            tmem_st32(tO + 32 * c, acc);
+          }
+        }
+        const bool zero_half[2] = {__all_sync(0xffffffffu, mx0 - m < SKIP_BELOW) != 0,
+                                   __all_sync(0xffffffffu, mx1 - m < SKIP_BELOW) != 0};
+        float lsum = 0.0f;
+        uint32_t ph[64];   // P as fp16 pairs: ph[c] = keys 2c (low), 2c + 1
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (zero_half[h]) {
+#pragma unroll
+            for (int c = 32 * h; c < 32 * h + 32; ++c) ph[c] = 0u;
+            continue;
+          }
+#pragma unroll
+          for (int c = 32 * h; c < 32 * h + 32; ++c) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), cs, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), cs, negm));
+            lsum += p0 + p1;
+            const __half2 h2 = __floats2half2_rn(p0, p1);
+            ph[c] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+        }
+        l = fmaf(l, alpha, lsum);
+        tmem_st32(tS + 64, ph);
+        tmem_st32(tS + 96, ph + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_PFULL + X]);
+      }
+      if (ok) ok = wait_all(B_ODONE + X, 0, 0x2102);
+      if (ok) {
+        // epilogue: O / l -> fp16 for rows < N; loads are warp-collective
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        const bool store = row < Pb.N;
+        __half* orow = o + ((size_t)bh * Pb.N + (store ? row : 0)) * D;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t acc[32];
+          tmem_ld32(tO + 32 * c, acc);
+          tmem_wait_ld();
+          uint32_t hv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __half2 h2 =
+                __floats2half2_rn(__uint_as_float(acc[2 * e]) * inv, __uint_as_float(acc[2 * e + 1]) * inv);
+            hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+          }
+        }
       }
     }
-  } else if (tid == 0) {
-    umma_commit(&bar[2]);
-    mbar_wait(&bar[2], 0, limit, err, 0x2003);
+  } else if (warp == 8 || warp == 11) {
+    // ------------------------------------------------------------ bulk copies (warp 8: Q, K; warp 11: V^T)
+    if (lane == 0) {
+      const bool isK = warp == 8;
+      const uint8_t* src = (isK ? kimg : vimg) + (size_t)bh * nt * 32768;
+      const int FULL = isK ? B_KFULL : B_VFULL, EMPTY = isK ? B_KEMPTY : B_VEMPTY;
+      const uint32_t base = isK ? Smem::K : Smem::V;
+      if (isK) {
+        const uint8_t* qsrc = qimg + ((size_t)bh * nt + qt0) * 32768;
+        mbar_expect_tx(&bar[B_QFULL], hasB ? 65536u : 32768u);
+        bulk_g2s(sm + Smem::QA, qsrc, 32768, &bar[B_QFULL]);
+        if (hasB) bulk_g2s(sm + Smem::QB, qsrc + 32768, 32768, &bar[B_QFULL]);
+      }
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % STAGES;
+        if (j >= STAGES &&
+            !mbar_wait_abortable(&bar[EMPTY + st], ((j / STAGES) - 1) & 1, abort_flag, limit, err, 0x2201))
+          break;
+        mbar_expect_tx(&bar[FULL + st], 32768u);
+        bulk_g2s(sm + base + st * 32768, src + (size_t)j * 32768, 32768, &bar[FULL + st]);
+        issued = j + 1;
+      }
+      if (*abort_flag) {   // let every copy still in flight land before the CTA exits
+        if (isK) mbar_wait(&bar[B_QFULL], 0, limit, err, 0x2203);
+        for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+          mbar_wait(&bar[FULL + j % STAGES], (j / STAGES) & 1, limit, err, 0x2204);
+      }
+    }
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    const int X = warp - 9;
+    if (lane == 0 && (X == 0 || hasB)) {
+      const uint32_t qa = smem_u32(sm + (X ? Smem::QB : Smem::QA));
+      const uint32_t kb = smem_u32(sm + Smem::K), vb = smem_u32(sm + Smem::V);
+      const uint32_t tS = tbase + X * 128, tO = tbase + 256 + X * 128;
+      auto wait = [&](int b, uint32_t parity, uint32_t site) {
+        return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
+      };
+      auto issue_S = [&](int j) {   // S_X(j) = Q_X K(j)^T, then release the K stage
+        const uint32_t kt = kb + (j % STAGES) * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) umma_f16(tS, desc(qa, kk), desc(kt, kk), IDESC, kk > 0);
+        umma_commit(&bar[B_SFULL + X]);
+        umma_commit(&bar[B_KEMPTY + j % STAGES]);
+      };
+      bool ok = wait(B_QFULL, 0, 0x2301) && wait(B_KFULL, 0, 0x2302);
+      if (ok) {
+        tc_fence_after();
+        issue_S(0);
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        if (!(ok = wait(B_PFULL + X, j & 1, 0x2303))) break;
+        if (!(ok = wait(B_VFULL + j % STAGES, (j / STAGES) & 1, 0x2304))) break;
+        tc_fence_after();
+        const uint32_t vt = vb + (j % STAGES) * 32768;   // O_X += P_X(j) V(j), P from TMEM
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_tmem_a(tO, tS + 64 + 8 * kk, desc(vt, kk), IDESC, (j > 0) || (kk > 0));
+        umma_commit(&bar[B_VEMPTY + j % STAGES]);
+        if (j + 1 < nt) {
+          if (!(ok = wait(B_KFULL + (j + 1) % STAGES, ((j + 1) / STAGES) & 1, 0x2305))) break;
+          tc_fence_after();
+          issue_S(j + 1);
+        } else {
+          umma_commit(&bar[B_ODONE + X]);
+        }
+      }
+      // every MMA this thread issued completes before TMEM is released
+      umma_commit(&bar[B_DRAIN + X]);
+      mbar_wait(&bar[B_DRAIN + X], 0, limit, err, 0x2308);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -210,13 +325,17 @@ __global__ void timeout_probe_kernel(WsHeader* hdr, uint64_t limit) {
 
 cudaError_t launch_fp16_attention(const Prob& p, __half* o, void* ws, cudaStream_t st) {
   const WsLayout L = ws_layout(p);
-  char* base = static_cast<char*>(ws);
-  const int smem = F16Smem::BYTES + 1024;
+  const uint8_t* base = static_cast<const uint8_t*>(ws);
+  const int smem = f16::Smem::BYTES + 1024;   // > half the SM: one CTA per SM owns all 512 TMEM columns
   cudaError_t e = cudaFuncSetAttribute(fp16_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fp16_attn_kernel<<<dim3(p.N_pad / TILE, p.BH), 128, smem, st>>>(
-      p, reinterpret_cast<const __half*>(base + L.qr), reinterpret_cast<const __half*>(base + L.kr),
-      reinterpret_cast<const __half*>(base + L.vt), o, static_cast<WsHeader*>(ws), wait_limit());
+  cudaFuncAttributes fa;   // the setmaxnreg split needs exactly LAUNCH_REGS at launch
+  e = cudaFuncGetAttributes(&fa, fp16_attn_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != f16::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+  const int nt = p.N_pad / TILE;
+  fp16_attn_kernel<<<dim3((nt + 1) / 2, p.BH), f16::NUM_THREADS, smem, st>>>(
+      p, base + L.qr, base + L.kr, base + L.vt, o, static_cast<WsHeader*>(ws), wait_limit());
   return cudaGetLastError();
 }
 

@@ -41,7 +41,8 @@ struct WsLayout {
   size_t img;                   // INT4 attention: INT8 operand images of Q, K, V^T,
                                 // 3 x [BH][N_pad / 128][16 KB]
   size_t base_bytes;            // end of the part the INT4 path needs
-  size_t qr, kr, vt;            // FP16 path: fp16 [BH][N_pad][128] x2, fp16 [BH][128][N_pad]
+  size_t qr, kr, vt;            // FP16 path: operand images of RoPE-encoded Q, K and of V^T,
+                                // [BH][N_pad / 128][32 KB] each (two swizzled 16 KB atoms)
   size_t total_fp16;
 };
 

@@ -262,9 +262,12 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const int c0 = 8 * g;
+  const int nt = P.N_pad / TILE;
   const __half* x = (which == 0 ? q : which == 1 ? k : v) + (size_t)bh * P.N * D;
   if (which < 2) {
-    __half* out = (which == 0 ? qr : kr) + (size_t)bh * P.N_pad * D;
+    // operand image: tile n / 128 is 32 KB, channels 0..63 and 64..127 in two
+    // 128-byte-swizzled K-major atoms of 16 KB
+    uint8_t* img = reinterpret_cast<uint8_t*>(which == 0 ? qr : kr) + (size_t)bh * nt * 32768;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int n = blk * QK_BLOCK + r0 + 8 * i;
@@ -277,7 +280,8 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
       }
-      *reinterpret_cast<uint4*>(out + (size_t)n * D + c0) = o;
+      *reinterpret_cast<uint4*>(img + (size_t)(n / TILE) * 32768 + (c0 >> 6) * 16384 +
+                                sw128_off(n % TILE, (c0 & 63) >> 3)) = o;
     }
     return;
   }
@@ -290,16 +294,17 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
     for (int e = 0; e < 8; ++e) tr[r][c0 + e] = h[e];
   }
   __syncthreads();
-  // thread c writes channel c's 64 tokens (128 bytes) of this block
+  // thread c writes channel c's 64 tokens (128 bytes) of this block: row c
+  // of the V^T operand image of key tile blk / 2, atom blk % 2
   const int c = threadIdx.x;
-  __half* dst = vt + ((size_t)bh * D + c) * P.N_pad + (size_t)blk * QK_BLOCK;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(vt) + ((size_t)bh * nt + blk / 2) * 32768 + (blk & 1) * 16384;
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     uint4 o;
     __half* h = reinterpret_cast<__half*>(&o);
 #pragma unroll
     for (int e = 0; e < 8; ++e) h[e] = tr[8 * t + e][c];
-    reinterpret_cast<uint4*>(dst)[t] = o;
+    *reinterpret_cast<uint4*>(dst + sw128_off(c, t)) = o;
   }
 }
 

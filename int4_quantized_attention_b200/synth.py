@@ -14,6 +14,10 @@ whose per-channel scale is shared by Q and K:
 * ``tiny``:  4 channels per RoPE segment (chosen per head) scaled by 8.
 * ``half``:  per-(head, channel) lognormal(0, 1) scale.
 * ``wan`` / ``hunyuan``: per-(head, channel) lognormal(0, 1.5) scale.
+* ``wan_flat``: a stress case, not one of the pages' workloads: the Wan
+  shapes with every Q/K channel scaled by 0.3, so the logits of a row stay
+  within about one unit of each other and almost every P code is non-zero
+  (no 64-key half of exponentials can be skipped).
 * V is N(0, 1) everywhere.
 
 Recipe (fixed, so that any consumer reproduces the same bytes):
@@ -70,6 +74,7 @@ CONFIGS = {
     "half": Config("half", 1, 4, 8, 16, 16, 0, (44, 42, 42), "half", "lognormal1", 102),
     "wan": Config("wan", 1, 40, 21, 45, 80, 0, (44, 42, 42), "interleaved", "lognormal1.5", 103),
     "hunyuan": Config("hunyuan", 1, 24, 33, 45, 80, 256, (16, 56, 56), "half", "lognormal1.5", 104),
+    "wan_flat": Config("wan_flat", 1, 40, 21, 45, 80, 0, (44, 42, 42), "interleaved", "const0.3", 105),
 }
 
 def _channel_scales(cfg: Config, rng: np.random.Generator) -> np.ndarray:
@@ -89,6 +94,8 @@ def _channel_scales(cfg: Config, rng: np.random.Generator) -> np.ndarray:
         return rng.lognormal(0.0, 1.5, size=(H, d)).astype(np.float32)
     if cfg.dist == "normal":
         return np.ones((H, d), np.float32)
+    if cfg.dist == "const0.3":
+        return np.full((H, d), 0.3, np.float32)
     raise ValueError(f"unknown distribution {cfg.dist!r}")
 
 
