@@ -276,7 +276,8 @@ def our_arm(args, cfg, rank, world):
         "vs_baseline": None, "dtype": "s8xs8->s32 (INT4 codes), fp32 softmax", "data": "synthetic",
         "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
                    "grid": [cfg.F, cfg.Hh, cfg.W], "n_text": cfg.n_text, "split": list(cfg.split),
-                   "rotation": cfg.rot, "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "rotation": cfg.rot, "p_mode": cfg.p_mode,
+                   "parallelism": "replicas" if world > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (q,k,v 2.3 GB; INT8 K/V operand images 0.77 GB per pass)"},
         "roofline": {"kernel": "int4_attn_kernel", "bound": "tensor", "achieved": attn_tops,
                      "peak": peak_int8, "unit": "TOPS", "frac": attn_tops / peak_int8, "traffic": profiled_traffic(cfg),
@@ -345,6 +346,8 @@ def main():
     ap.add_argument("--schedule", action="store_true", help="also run the 400-call mixed schedule")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
+    ap.add_argument("--p-mode", default="range", choices=["range", "symmetric"],
+                    help="P quantisation of the INT4 path (range-optimised: the method)")
     ap.add_argument("--only-step", action="store_true",
                     help="run only the warm-up and timed INT4 steps (for profiler captures)")
     args = ap.parse_args()
@@ -352,6 +355,8 @@ def main():
     cfg = synth.CONFIGS[args.config]
     if args.heads:
         cfg = cfg.replace(H=args.heads, name=f"{cfg.name}-H{args.heads}")
+    if args.p_mode != "range":
+        cfg = cfg.replace(p_mode=args.p_mode, name=f"{cfg.name}-p{args.p_mode}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

@@ -49,6 +49,19 @@ typedef enum {
     RA_ROT_HALF = 2             /* H2 on (i, i + d_s/2) in each segment (Fig. 3) */
 } ra_rot_mode;
 
+/* Quantisation of P = exp(s - m) in [0, 1] for the P.V product.
+ * RA_P_RANGE_OPTIMIZED (the method): code = rne(15 P) - 8 in [-8, 7], the
+ *   full signed INT4 range, with the zero-point corrected through the V
+ *   column sums ("What carries the argument"; free-parameter ledger, Sec. 4.2).
+ * RA_P_SYMMETRIC: plain symmetric INT4, code = rne(7 P) in [0, 7], no
+ *   zero-point (the baseline that leaves half the codes unused, abstract); the
+ *   pages' referee report and the "If this is right" list suggest disabling
+ *   the range-optimised map for low-entropy (image-to-video) attention. */
+typedef enum {
+    RA_P_RANGE_OPTIMIZED = 0,
+    RA_P_SYMMETRIC = 1
+} ra_p_mode;
+
 /* One attention problem.  Tokens: N = F*Hh*W video tokens in frame-major
  * order (frame slowest, column fastest) followed by n_text text tokens, which
  * get no RoPE but do get the rotation.  head_dim d is split into three RoPE
@@ -60,6 +73,7 @@ typedef struct {
     int split[3];
     double theta;               /* RoPE base, e.g. 10000.0 */
     int rot;                    /* ra_rot_mode */
+    int p_mode;                 /* ra_p_mode (INT4 attention only; 0 = the method) */
 } ra_problem;
 
 /* Quantised Q, K, V as produced by ra_rotate_quantize_qkv (device memory).

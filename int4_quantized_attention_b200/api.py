@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "librotate_attn.so")
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_WORKSPACE, RA_ERR_CUDA, \
     RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(7)
 ROT = {"none": 0, "interleaved": 1, "half": 2}
+P_MODE = {"range": 0, "symmetric": 1}       # ra_p_mode
 
 
 class RotateAttnError(RuntimeError):
@@ -30,7 +31,7 @@ class Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("n_text", ctypes.c_int), ("split", ctypes.c_int * 3),
-                ("theta", ctypes.c_double), ("rot", ctypes.c_int)]
+                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("p_mode", ctypes.c_int)]
 
 
 class Qkv4(ctypes.Structure):
@@ -102,6 +103,7 @@ def problem(cfg, rot: Optional[str] = None) -> Problem:
     p.split = (ctypes.c_int * 3)(*cfg.split)
     p.theta = float(cfg.theta)
     p.rot = ROT[rot if rot is not None else cfg.rot]
+    p.p_mode = P_MODE[getattr(cfg, "p_mode", "range")]
     return p
 
 

@@ -39,7 +39,8 @@
 // are exactly the float 1.5 * 2^23 + 256 S: the softmax takes its row max and
 // its exponent arguments on the raw bits, with no integer-to-float step.
 //
-// The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15], fed as an
+// The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15] (with the
+// symmetric P map instead: w = rne(7 * 2^(x - m)) = code), fed as an
 // unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
 // sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
 // The int32 P.V accumulator stays in TMEM across tiles; the rescale is an
@@ -232,6 +233,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       {
         const int grow = (qt0 + X) * TILE + (int)row;
         const float kq = __fmul_rn(a.sq[(size_t)bh * nblk + grow / QK_BLOCK], LOG2E / (SQRT_D * 256.0f));
+        // P map: w = rne(pscale * P); range-optimised: pscale 15, code = w - 8;
+        // symmetric: pscale 7, code = w.  w = 0 wherever pscale * 2^x <= 1/2,
+        // i.e. x <= log2(1 / (2 pscale)) (-4.91 and -3.81): skip_below lies under it.
+        const float pscale = P.p_mode == RA_P_SYMMETRIC ? 7.0f : 15.0f;
+        const float skip_below = P.p_mode == RA_P_SYMMETRIC ? -4.0f : -5.0f;
+        const int zp = P.p_mode == RA_P_SYMMETRIC ? 0 : 8;
         const float* skb = a.sk + (size_t)bh * nblk;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const uint32_t tS = tbase + X * 128 + lane_off, tO = tbase + 256 + X * 128 + lane_off;
@@ -288,8 +295,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
           // 64-key half whose largest x is below -5 holds only zero codes.
           // Skip its exponentials when that is so for every row of the warp.
-          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < -5.0f) != 0,
-                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < -5.0f) != 0};
+          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < skip_below) != 0,
+                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < skip_below) != 0};
           uint32_t L = 0;
           uint32_t pw[32];
 #pragma unroll
@@ -306,7 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               for (int e = 0; e < 8; ++e) {
                 const int n = 4 * k + e;
                 const float x = fmaf(__int_as_float(s[n]) - MAGIC, h ? c1 : c0, negm);
-                wb[e] = __float_as_uint(fmaf(15.0f, ex2(x), MAGIC));   // low byte = w
+                wb[e] = __float_as_uint(fmaf(pscale, ex2(x), MAGIC));   // low byte = w
               }
               const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
               const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
 #pragma unroll
             for (int n = 0; n < 128; ++n) {
               const int w = (int)((pw[2 * (n >> 3) + (n & 1)] >> (8 * ((n & 7) >> 1))) & 0xFF);
-              a.dbg_p[row * TILE + n] = n < nvalid ? (int8_t)(w - 8) : (int8_t)-128;
+              a.dbg_p[row * TILE + n] = n < nvalid ? (int8_t)(w - zp) : (int8_t)-128;
             }
           }
           tc_fence_before();

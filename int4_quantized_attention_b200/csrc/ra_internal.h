@@ -24,6 +24,7 @@ struct Prob {
   int tab_off[3];               // first table entry of each segment
   int n_tab;                    // table entries (each: cos, sin, alpha, beta)
   int rot;
+  int p_mode;                   // ra_p_mode
   uint64_t signature;
 };
 

@@ -53,6 +53,7 @@ class Config:
     seed: int
     d: int = D_HEAD
     theta: float = 10000.0
+    p_mode: str = "range"    # P quantisation: "range" (the method) | "symmetric"
 
     @property
     def N(self) -> int:

@@ -55,6 +55,8 @@ def lib():
         _lib = ctypes.CDLL(build_oracle())
         _lib.orc_p_code.restype = ctypes.c_int
         _lib.orc_p_code.argtypes = [ctypes.c_float]
+        _lib.orc_p_code_sym.restype = ctypes.c_int
+        _lib.orc_p_code_sym.argtypes = [ctypes.c_float]
         _lib.orc_rope_angle.restype = ctypes.c_double
         _lib.orc_seq_len.restype = ctypes.c_int
         _lib.orc_seq_pad.restype = ctypes.c_int
@@ -101,6 +103,17 @@ def rope_angle(cfg, s: int, pos: int, j: int) -> float:
 
 def p_code(P: float) -> int:
     return lib().orc_p_code(ctypes.c_float(P))
+
+
+def p_code_sym(P: float) -> int:
+    return lib().orc_p_code_sym(ctypes.c_float(P))
+
+
+def _quant_mode(cfg, quant_p) -> int:
+    """0: exact P; 1: range-optimised P code; 2: symmetric P code."""
+    if not quant_p:
+        return 0
+    return 2 if getattr(cfg, "p_mode", "range") == "symmetric" else 1
 
 
 def rotate_head(cfg, x: np.ndarray, rot: Optional[str] = None) -> np.ndarray:
@@ -156,7 +169,7 @@ def attention_rows(cfg, qz: dict, rows=None, tile: int = 128, quant_p: bool = Tr
     rows = np.arange(cfg.N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
     out = np.empty((len(rows), cfg.d), np.float16)
     out64 = np.empty((len(rows), cfg.d), np.float64) if want64 else None
-    lib().orc_attention_rows(ctypes.byref(problem(cfg)), _ptr(rows), len(rows), tile, int(quant_p),
+    lib().orc_attention_rows(ctypes.byref(problem(cfg)), _ptr(rows), len(rows), tile, _quant_mode(cfg, quant_p),
                              _ptr(qz["qc"]), _ptr(qz["qs"]), _ptr(qz["kc"]), _ptr(qz["ks"]),
                              _ptr(qz["vc"]), _ptr(qz["sv"]), _ptr(qz["colsum"]), _ptr(out),
                              _ptr(out64) if want64 else None)
@@ -168,7 +181,7 @@ def attention_row_debug(cfg, qz: dict, i: int, tile_index: int, tile: int = 128)
     S = np.zeros((tile,), np.int32)
     P = np.zeros((tile,), np.int8)
     o = np.empty((cfg.d,), np.float16)
-    lib().orc_attention_row(ctypes.byref(problem(cfg)), i, tile, 1,
+    lib().orc_attention_row(ctypes.byref(problem(cfg)), i, tile, _quant_mode(cfg, True),
                             _ptr(qz["qc"]), _ptr(qz["qs"]), _ptr(qz["kc"]), _ptr(qz["ks"]),
                             _ptr(qz["vc"]), _ptr(qz["sv"]), _ptr(qz["colsum"]), _ptr(o), None,
                             tile_index, _ptr(S), _ptr(P))

@@ -244,6 +244,12 @@ void orc_quantize_v_head(const orc_problem *p, const f16 *v, int8_t *codes, floa
  * (fixed scale 15, zero-point -8; Sec. 4.2). */
 int orc_p_code(float P) { return (int)nearbyintf(15.0f * P) - 8; }
 
+/* Symmetric INT4 code of P in [0,1] (the map the range-optimised one
+ * replaces; abstract: symmetric quantisation of the non-negative P leaves
+ * half of the codes unused): scale max|P| / 7 = 1/7, code = rne(7 P) in [0, 7],
+ * no zero-point. */
+int orc_p_code_sym(float P) { return (int)nearbyintf(7.0f * P); }
+
 /* One query row i of the INT4 attention (one head), T_kv = `tile` keys per
  * step of the online softmax (128 for the method as built).
  *
@@ -260,6 +266,8 @@ int orc_p_code(float P) { return (int)nearbyintf(15.0f * P) - 8; }
  * logits; the normaliser uses the dequantised codes (keeps O a convex
  * combination of dequantised V rows); P is quantised against the running max.
  *
+ * quant_p = 1: the range-optimised code above.  quant_p = 2: the symmetric
+ * code rne(7 P) instead, with no zero-point term and L = sum code.
  * quant_p = 0 replaces the P code by the exact P (float64) and drops the
  * zero-point, for checking the loop against two-pass softmax attention.
  * Optional outputs: o64 [d] (float64 before the fp16 rounding); for tile
@@ -299,16 +307,18 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
         if (quant_p) {
             int64_t pvi[512] = {0};
             int64_t Li = 0;
+            const int zp = quant_p == 2 ? 0 : 8;
             for (int n = n0; n < n1; ++n) {
                 float P = expf(sl[n - n0] - m_new);
-                int code = orc_p_code(P);
-                Li += code + 8;
+                int code = quant_p == 2 ? orc_p_code_sym(P) : orc_p_code(P);
+                Li += code + zp;
                 for (int c = 0; c < d; ++c) pvi[c] += (int64_t)code * vc[(size_t)n * d + c];
                 if (j == dbg_tile && dbg_P) dbg_P[n - n0] = (int8_t)code;
             }
             /* zero-point correction: + 8 * sum over the tile's keys of the V codes */
-            for (int g = n0 / QK_BLOCK; g * QK_BLOCK < n1; ++g)
-                for (int c = 0; c < d; ++c) pvi[c] += 8 * (int64_t)colsum[(size_t)g * d + c];
+            if (zp)
+                for (int g = n0 / QK_BLOCK; g * QK_BLOCK < n1; ++g)
+                    for (int c = 0; c < d; ++c) pvi[c] += 8 * (int64_t)colsum[(size_t)g * d + c];
             for (int c = 0; c < d; ++c) pv[c] = (double)pvi[c];
             L = (double)Li;
         } else {

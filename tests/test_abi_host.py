@@ -49,6 +49,10 @@ def test_validation_codes(lib):
     assert api.validate(prob(split=(43, 43, 42))) == api.RA_ERR_INVALID_ARG   # odd
     assert api.validate(prob(F=0, Hh=0, W=0, n_text=0)) == api.RA_ERR_INVALID_ARG   # N = 0
     assert api.validate(prob(H=0)) == api.RA_ERR_INVALID_ARG
+    assert api.validate(prob(p_mode="symmetric")) == api.RA_OK
+    bad = prob()
+    bad.p_mode = 2                                                           # unknown P map
+    assert api.validate(bad) == api.RA_ERR_INVALID_ARG
     assert api.validate(prob(theta=0.0)) == api.RA_ERR_INVALID_ARG
     p = prob()
     p.rot = 7

@@ -83,6 +83,10 @@ SMALL = {
     "text_only": synth.Config("text_only", 1, 1, 0, 0, 0, 130, (44, 42, 42), "half", "outlier8", 14),
     # several tiles: N = 4*16*20 = 1280
     "multi_tile": synth.Config("multi_tile", 1, 2, 4, 16, 20, 0, (44, 42, 42), "interleaved", "lognormal1.5", 15),
+    # the symmetric P map (RA_P_SYMMETRIC) on a half-rotation and a ragged case
+    "half_sym": synth.CONFIGS["half"].replace(name="half_sym", p_mode="symmetric"),
+    "ragged_sym": synth.Config("ragged_sym", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 16,
+                               p_mode="symmetric"),
 }
 
 
@@ -105,7 +109,8 @@ def test_int4_path_matches_oracle(oracle_mod, dev, name):
     assert worst_err <= MAXABS_INT4, worst_err
 
 
-@pytest.mark.parametrize("name", ["tiny", "half", "ragged_text", "text_only", "multi_tile"])
+@pytest.mark.parametrize("name", ["tiny", "half", "ragged_text", "text_only", "multi_tile", "half_sym",
+                                  "ragged_sym"])
 def test_int4_S_tiles_bit_exact_and_P_codes(oracle_mod, dev, name):
     cfg = SMALL[name]
     q, k, v = synth.make_qkv(cfg)

@@ -45,6 +45,23 @@ def test_p_map_golden(oracle_mod):
     assert np.max(np.abs((codes - g["zero_point"]) / g["scale"] - grid)) <= 1.0 / 30 + 1e-7
 
 
+def test_p_map_symmetric_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "p_map_symmetric.json")))
+    for P, code in g["endpoints"]:
+        assert oracle_mod.p_code_sym(P) == code
+    lo, hi = g["code_range"]
+    for kk in range(8):
+        assert oracle_mod.p_code_sym(np.float32(kk) / np.float32(g["scale"])) == kk + g["zero_point"]
+    grid = np.linspace(0.0, 1.0, 20001, dtype=np.float32)
+    codes = np.array([oracle_mod.p_code_sym(float(x)) for x in grid])
+    assert codes.min() == lo and codes.max() == hi
+    assert np.all(np.diff(codes) >= 0)
+    # half a step of the symmetric map is 1/14: twice the range-optimised 1/30
+    assert np.max(np.abs(codes / g["scale"] - grid)) <= 1.0 / 14 + 1e-7
+    # round half to even at the step midpoints, like the range-optimised map
+    assert oracle_mod.p_code_sym(0.5 / 7) == 0 and oracle_mod.p_code_sym(1.5 / 7) == 2
+
+
 def test_schedule_golden():
     g = json.load(open(os.path.join(GOLDEN, "schedule.json")))
     for c in g["cases"]:
@@ -312,6 +329,27 @@ def test_zero_point_identity_single_tile(oracle_mod):
         ref = (w @ qz["vc"][:128].astype(np.int64)) * qz["sv"].astype(np.float64) / w.sum()
         assert np.allclose(o64[i], ref, rtol=1e-12, atol=1e-12)
         assert w.max() == 15                               # the row max always gets P = 1
+
+
+def test_symmetric_p_single_tile_and_error_bound(oracle_mod):
+    """Symmetric P map: within one tile O = sum code * v / sum code (no
+    zero-point term), the row max gets code 7, and every code is within half
+    a step (1/14) of exp(s - m) (numpy, float64)."""
+    cfg = small_cfg(F=2, Hh=8, W=8, rot="interleaved", p_mode="symmetric")   # N = 128: one tile
+    _, _, _, qz = random_qz(oracle_mod, cfg, 8, qscale=1.5)
+    _, o64 = oracle_mod.attention_rows(cfg, qz, want64=True)
+    _, s = dequant_logits(cfg, qz)
+    for i in (0, 17, 127):
+        _, P = oracle_mod.attention_row_debug(cfg, qz, i, 0)
+        w = P.astype(np.int64)
+        assert w.min() >= 0 and w.max() == 7
+        ref = (w @ qz["vc"][:128].astype(np.int64)) * qz["sv"].astype(np.float64) / w.sum()
+        assert np.allclose(o64[i], ref, rtol=1e-12, atol=1e-12)
+        assert np.max(np.abs(w / 7.0 - np.exp(s[i, :128] - s[i, :128].max()))) <= 1 / 14 + 1e-6
+    # the two maps differ on the same inputs (the range-optimised one is finer)
+    o_range = oracle_mod.attention_rows(cfg.replace(p_mode="range"), qz)
+    o_sym = oracle_mod.attention_rows(cfg, qz)
+    assert not np.array_equal(o_range, o_sym)
 
 
 def test_uniform_logits_give_the_mean(oracle_mod):
