@@ -171,6 +171,23 @@ def reference_arm(args, cfg, rank):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest per-rank value (each rank's device time): the whole job
+    is as slow as its slowest replica.  A no-op for one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tops(world: int, ops_per_replica: float, ms: float) -> float:
+    """Whole-job throughput: every replica does ops_per_replica in ms."""
+    return world * ops_per_replica / (ms * 1e-3) / 1e12
+
+
 def event_time(fn, iters, stream):
     import torch
     start = torch.cuda.Event(enable_timing=True)
@@ -223,10 +240,8 @@ def our_arm(args, cfg, rank, world):
             print(json.dumps({"workload": cfg.name, "ms_per_step": ms_step, "int4_attention_ms": ms_attn,
                               "prologue_ms": ms_pro}), flush=True)
         return
+    ms_step = max_over_ranks(ms_step, dev)
     if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
         dist.barrier()
 
     # FP16 path on the same workload (a few calls)
@@ -247,10 +262,7 @@ def our_arm(args, cfg, rank, world):
     e2e_step()
     ms_e2e = event_time(e2e_step, max(2, args.steps // 2), stream)
     ra.check()
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dev)
 
     sched = None
     if args.schedule:
@@ -259,7 +271,7 @@ def our_arm(args, cfg, rank, world):
     if rank != 0:
         return
     ops = cfg.ops
-    tops = world * ops / (ms_step * 1e-3) / 1e12
+    tops = aggregate_tops(world, ops, ms_step)
     attn_tops = ops / (ms_attn * 1e-3) / 1e12
     # the attention kernel is timed alone: burst GEMM figure x the int8:bf16 ratio
     peak_int8 = peaks["bf16"] * INT8_PER_BF16
@@ -294,7 +306,7 @@ def our_arm(args, cfg, rank, world):
                       "frac_bf16_peak_sustained": ops / (ms_f16 * 1e-3) / 1e12 / peaks["bf16_sus"],
                       "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TF/s (the call is timed alone)",
                       "int4_step_speedup": ms_f16 / ms_step},
-        "e2e": {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
+        "e2e": {"value": aggregate_tops(world, ops, ms_e2e), "unit": "TOPS", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
