@@ -358,6 +358,8 @@ def main():
     ap.add_argument("--schedule", action="store_true", help="also run the 400-call mixed schedule")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
+    ap.add_argument("--rot", default=None, choices=["none", "interleaved", "half", "full"],
+                    help="override the workload's rotation mode")
     ap.add_argument("--p-mode", default="range", choices=["range", "symmetric"],
                     help="P quantisation of the INT4 path (range-optimised: the method)")
     ap.add_argument("--only-step", action="store_true",
@@ -367,6 +369,8 @@ def main():
     cfg = synth.CONFIGS[args.config]
     if args.heads:
         cfg = cfg.replace(H=args.heads, name=f"{cfg.name}-H{args.heads}")
+    if args.rot is not None and args.rot != cfg.rot:
+        cfg = cfg.replace(rot=args.rot, name=f"{cfg.name}-r{args.rot}")
     if args.p_mode != "range":
         cfg = cfg.replace(p_mode=args.p_mode, name=f"{cfg.name}-p{args.p_mode}")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -46,7 +46,13 @@ typedef enum {
 typedef enum {
     RA_ROT_NONE = 0,            /* RoPE only */
     RA_ROT_INTERLEAVED = 1,     /* H2 on adjacent dims, merged into RoPE (Fig. 3) */
-    RA_ROT_HALF = 2             /* H2 on (i, i + d_s/2) in each segment (Fig. 3) */
+    RA_ROT_HALF = 2,            /* H2 on (i, i + d_s/2) in each segment (Fig. 3) */
+    RA_ROT_FULL = 3             /* dense rotation over all of head_dim after RoPE: the
+                                 * normalised 128-point Walsh-Hadamard transform (the
+                                 * "Full" rotation the pages compare against, Figs. 4-5;
+                                 * the matrix is not given there).  Computed as the fast
+                                 * transform in fp32, strides 1, 2, ..., 64, then one
+                                 * multiply by fp32(1/sqrt(128)). */
 } ra_rot_mode;
 
 /* Quantisation of P = exp(s - m) in [0, 1] for the P.V product.

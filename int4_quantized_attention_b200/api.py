@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(PKG, "librotate_attn.so")
 
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_WORKSPACE, RA_ERR_CUDA, \
     RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(7)
-ROT = {"none": 0, "interleaved": 1, "half": 2}
+ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3}
 P_MODE = {"range": 0, "symmetric": 1}       # ra_p_mode
 
 

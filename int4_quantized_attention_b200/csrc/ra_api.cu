@@ -61,7 +61,7 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     sum += p->split[s];
   }
   if (sum != p->d) return fail(RA_ERR_INVALID_ARG, "RoPE split sums to %d, head_dim is %d", sum, p->d);
-  if (p->rot != RA_ROT_NONE && p->rot != RA_ROT_INTERLEAVED && p->rot != RA_ROT_HALF)
+  if (p->rot != RA_ROT_NONE && p->rot != RA_ROT_INTERLEAVED && p->rot != RA_ROT_HALF && p->rot != RA_ROT_FULL)
     return fail(RA_ERR_INVALID_ARG, "rotation mode %d unknown", p->rot);
   if (!(p->theta > 0.0) || !std::isfinite(p->theta)) return fail(RA_ERR_INVALID_ARG, "RoPE base must be > 0");
   if (p->p_mode != RA_P_RANGE_OPTIMIZED && p->p_mode != RA_P_SYMMETRIC)

@@ -20,6 +20,7 @@ namespace ra {
 namespace {
 
 constexpr float kRsqrt2 = 0.70710678118654752440f;   // fp32 rounding of 1/sqrt(2)
+constexpr float kRsqrt128 = 0.08838834764831844055f; // fp32 rounding of 1/sqrt(128)
 
 struct TokenPos {
   int p[3];
@@ -148,6 +149,34 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
         const float b = first ? ys[r][c + h] : ys[r][c];
         z[i][e] = first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
       }
+    }
+  }
+  if (ROT == RA_ROT_FULL) {
+    // normalised 128-point Walsh-Hadamard transform of every row, strides
+    // 1, 2, 4 inside a thread's 8 channels, 8 .. 64 across the 16 lanes that
+    // hold the row (lane bit h / 8); pair (k, k + h) -> (a + b, a - b)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+      for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (!(e & h)) {
+            const float a = z[i][e], b = z[i][e + h];
+            z[i][e] = __fadd_rn(a, b);
+            z[i][e + h] = __fsub_rn(a, b);
+          }
+#pragma unroll
+      for (int hl = 1; hl < 16; hl <<= 1) {
+        const bool upper = (g & hl) != 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float other = __shfl_xor_sync(0xffffffffu, z[i][e], hl);
+          z[i][e] = upper ? __fsub_rn(other, z[i][e]) : __fadd_rn(z[i][e], other);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[i][e] = __fmul_rn(z[i][e], kRsqrt128);
     }
   }
 #pragma unroll
@@ -324,6 +353,7 @@ cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, con
     case RA_ROT_INTERLEAVED:
       qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
       break;
+    case RA_ROT_FULL: qk_quant_kernel<RA_ROT_FULL><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
     default: qk_quant_kernel<RA_ROT_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
   }
   cudaError_t e = cudaGetLastError();

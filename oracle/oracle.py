@@ -17,7 +17,7 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "rotate_attn_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
-ROT = {"none": 0, "interleaved": 1, "half": 2}
+ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3}
 
 
 def compile_oracle(src: str, out: str) -> None:

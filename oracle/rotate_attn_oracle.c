@@ -46,7 +46,7 @@ typedef struct {
     int rot;              /* 0 = no rotation, 1 = Interleaved, 2 = Half */
 } orc_problem;
 
-enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2 };
+enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2, ORC_ROT_FULL = 3 };
 enum { QK_BLOCK = 64, KV_TILE = 128 };
 
 int orc_seq_len(const orc_problem *p) { return p->F * p->Hh * p->W + p->n_text; }
@@ -145,6 +145,24 @@ void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
     rope_row(p, n, x, y);
     if (p->rot == ORC_ROT_NONE) {
         memcpy(z, y, sizeof(float) * p->d);
+        return;
+    }
+    if (p->rot == ORC_ROT_FULL) {
+        /* "Full" rotation (the dense comparison of Figs. 4-5; READING: the
+         * normalised Walsh-Hadamard matrix H/sqrt(d), Sylvester order, as the
+         * fast transform: for h = 1, 2, ..., d/2 every pair (k, k + h) with
+         * k & h == 0 becomes (a + b, a - b) in fp32; then one multiply by
+         * fp32(1/sqrt(d)). */
+        int d = p->d;
+        for (int h = 1; h < d; h <<= 1)
+            for (int i = 0; i < d; i += 2 * h)
+                for (int k = i; k < i + h; ++k) {
+                    float a = y[k], b = y[k + h];
+                    y[k] = a + b;
+                    y[k + h] = a - b;
+                }
+        const float r = (float)(1.0 / sqrt((double)d));
+        for (int c = 0; c < d; ++c) z[c] = y[c] * r;
         return;
     }
     const float r = (float)M_SQRT1_2;

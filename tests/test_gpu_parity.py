@@ -83,6 +83,8 @@ SMALL = {
     "text_only": synth.Config("text_only", 1, 1, 0, 0, 0, 130, (44, 42, 42), "half", "outlier8", 14),
     # several tiles: N = 4*16*20 = 1280
     "multi_tile": synth.Config("multi_tile", 1, 2, 4, 16, 20, 0, (44, 42, 42), "interleaved", "lognormal1.5", 15),
+    # the Full (128-point Walsh-Hadamard) rotation, ragged, with text tokens
+    "full_rot": synth.Config("full_rot", 1, 2, 3, 8, 10, 9, (44, 42, 42), "full", "lognormal1.5", 17),
     # the symmetric P map (RA_P_SYMMETRIC) on a half-rotation and a ragged case
     "half_sym": synth.CONFIGS["half"].replace(name="half_sym", p_mode="symmetric"),
     "ragged_sym": synth.Config("ragged_sym", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 16,

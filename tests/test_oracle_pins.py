@@ -136,7 +136,7 @@ def test_rope_rotates_pairs_counterclockwise(oracle_mod):
             assert np.count_nonzero(z) <= 2
 
 
-@pytest.mark.parametrize("rot", ["none", "interleaved", "half"])
+@pytest.mark.parametrize("rot", ["none", "interleaved", "half", "full"])
 def test_rope_relative_position(oracle_mod, rot):
     """q(p+D).k(p'+D) == q(p).k(p'): only the offset along each axis matters."""
     cfg = small_cfg(F=4, Hh=5, W=6, rot=rot)
@@ -195,7 +195,7 @@ def test_half_pairs_opposite_half_segments(oracle_mod):
             assert z[off + i + h] == pytest.approx(-r, abs=1e-7)
 
 
-@pytest.mark.parametrize("rot", ["interleaved", "half"])
+@pytest.mark.parametrize("rot", ["interleaved", "half", "full"])
 @pytest.mark.parametrize("split", [(44, 42, 42), (16, 56, 56)])
 def test_rotation_is_orthogonal(oracle_mod, rot, split):
     """QR.(KR)^T == QK^T and |xR| == |x| (the paper's orthogonality argument)."""
@@ -214,9 +214,27 @@ def test_rotation_is_orthogonal(oracle_mod, rot, split):
     assert np.max(np.abs(zq - yq)) > 0.1
 
 
+def test_full_rotation_is_the_normalised_hadamard(oracle_mod):
+    """Full rotation == RoPE output times H/sqrt(128), H the Sylvester
+    Hadamard matrix (scipy), in float64, to fp32 rounding."""
+    from scipy.linalg import hadamard
+    cfg = small_cfg(F=2, Hh=3, W=4, n_text=2)
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((cfg.N, 128)) * 2).astype(np.float16)
+    y = oracle_mod.rotate_head(cfg, x, rot="none").astype(np.float64)
+    z = oracle_mod.rotate_head(cfg.replace(rot="full"), x).astype(np.float64)
+    ref = y @ (hadamard(128).astype(np.float64) / math.sqrt(128))
+    assert np.max(np.abs(z - ref)) <= 4e-6 * np.max(np.abs(ref))
+    # a single channel spreads evenly over all 128 outputs
+    e = np.zeros((1, 128), np.float16)
+    e[0, 5] = 1
+    zz = oracle_mod.rotate_head(small_cfg(F=0, Hh=0, W=0, n_text=1, rot="full"), e)
+    assert np.allclose(np.abs(zz), 1 / math.sqrt(128), rtol=1e-6)
+
+
 # ---------------------------------------------------------------- quantisers
 
-@pytest.mark.parametrize("rot", ["interleaved", "half"])
+@pytest.mark.parametrize("rot", ["interleaved", "half", "full"])
 def test_qk_quantiser_properties(oracle_mod, rot):
     cfg = small_cfg(F=2, Hh=10, W=10, n_text=16, rot=rot)     # N = 216: ragged 64-blocks
     rng = np.random.default_rng(3)
