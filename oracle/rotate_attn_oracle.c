@@ -161,7 +161,7 @@ void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
                     y[k] = a + b;
                     y[k + h] = a - b;
                 }
-        const float r = (float)(1.0 / sqrt((double)d));
+        const float r = (float)(1.0 / sqrt((double)p->d));
         for (int c = 0; c < d; ++c) z[c] = y[c] * r;
         return;
     }
