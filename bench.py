@@ -288,7 +288,7 @@ def our_arm(args, cfg, rank, world):
         "vs_baseline": None, "dtype": "s8xs8->s32 (INT4 codes), fp32 softmax", "data": "synthetic",
         "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
                    "grid": [cfg.F, cfg.Hh, cfg.W], "n_text": cfg.n_text, "split": list(cfg.split),
-                   "rotation": cfg.rot, "p_mode": cfg.p_mode,
+                   "rotation": cfg.rot, "p_mode": cfg.p_mode, "v_rot": cfg.v_rot,
                    "parallelism": "replicas" if world > 1 else "single-gpu",
                    "l2": "inputs larger than L2 (q,k,v 2.3 GB; INT8 K/V operand images 0.77 GB per pass)"},
         "roofline": {"kernel": "int4_attn_kernel", "bound": "tensor", "achieved": attn_tops,
@@ -360,6 +360,7 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
     ap.add_argument("--rot", default=None, choices=["none", "interleaved", "half", "full"],
                     help="override the workload's rotation mode")
+    ap.add_argument("--v-rot", action="store_true", help="Hadamard on V inside the INT4 path (undone on O)")
     ap.add_argument("--p-mode", default="range", choices=["range", "symmetric"],
                     help="P quantisation of the INT4 path (range-optimised: the method)")
     ap.add_argument("--only-step", action="store_true",
@@ -371,6 +372,8 @@ def main():
         cfg = cfg.replace(H=args.heads, name=f"{cfg.name}-H{args.heads}")
     if args.rot is not None and args.rot != cfg.rot:
         cfg = cfg.replace(rot=args.rot, name=f"{cfg.name}-r{args.rot}")
+    if args.v_rot:
+        cfg = cfg.replace(v_rot=1, name=f"{cfg.name}-vrot")
     if args.p_mode != "range":
         cfg = cfg.replace(p_mode=args.p_mode, name=f"{cfg.name}-p{args.p_mode}")
     world = int(os.environ.get("WORLD_SIZE", "1"))

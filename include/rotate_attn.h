@@ -80,6 +80,11 @@ typedef struct {
     double theta;               /* RoPE base, e.g. 10000.0 */
     int rot;                    /* ra_rot_mode */
     int p_mode;                 /* ra_p_mode (INT4 attention only; 0 = the method) */
+    int v_rot;                  /* 1: the INT4 path multiplies every V row by the
+                                 * normalised 128-point Walsh-Hadamard matrix before
+                                 * quantising it and every output row by its transpose
+                                 * (a stand-in for the Hadamard the pages fuse into V
+                                 * offline: review page summary); 0: V as given */
 } ra_problem;
 
 /* Quantised Q, K, V as produced by ra_rotate_quantize_qkv (device memory).

@@ -31,7 +31,8 @@ class Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("n_text", ctypes.c_int), ("split", ctypes.c_int * 3),
-                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("p_mode", ctypes.c_int)]
+                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("p_mode", ctypes.c_int),
+                ("v_rot", ctypes.c_int)]
 
 
 class Qkv4(ctypes.Structure):
@@ -104,6 +105,7 @@ def problem(cfg, rot: Optional[str] = None) -> Problem:
     p.theta = float(cfg.theta)
     p.rot = ROT[rot if rot is not None else cfg.rot]
     p.p_mode = P_MODE[getattr(cfg, "p_mode", "range")]
+    p.v_rot = int(getattr(cfg, "v_rot", 0))
     return p
 
 

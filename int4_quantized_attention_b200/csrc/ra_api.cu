@@ -66,6 +66,7 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
   if (!(p->theta > 0.0) || !std::isfinite(p->theta)) return fail(RA_ERR_INVALID_ARG, "RoPE base must be > 0");
   if (p->p_mode != RA_P_RANGE_OPTIMIZED && p->p_mode != RA_P_SYMMETRIC)
     return fail(RA_ERR_INVALID_ARG, "P quantisation mode %d unknown", p->p_mode);
+  if (p->v_rot != 0 && p->v_rot != 1) return fail(RA_ERR_INVALID_ARG, "v_rot must be 0 or 1, not %d", p->v_rot);
   const long long Np = (N + ra::TILE - 1) / ra::TILE * ra::TILE;
   if (Np * ra::D >= (1ll << 31)) return fail(RA_ERR_UNSUPPORTED, "sequence too long: %lld tokens", N);
   if ((long long)p->B * p->H > 65535) return fail(RA_ERR_UNSUPPORTED, "B*H > 65535");
@@ -82,6 +83,7 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     P.W = p->W;
     P.rot = p->rot;
     P.p_mode = p->p_mode;
+    P.v_rot = p->v_rot;
     const int npos[3] = {p->F > 0 ? p->F : 1, p->Hh > 0 ? p->Hh : 1, p->W > 0 ? p->W : 1};
     int off = 0, toff = 0;
     for (int s = 0; s < 3; ++s) {

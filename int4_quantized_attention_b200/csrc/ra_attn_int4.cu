@@ -382,6 +382,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const float* svb = a.sv + (size_t)bh * D;
           const bool store = grow < P.N && !dbg_run;
           __half* orow = a.o + ((size_t)bh * P.N + (store ? grow : 0)) * D;
+          if (P.v_rot) {
+            // V was quantised as V H / sqrt(128): the row O' = O H / sqrt(128)
+            // goes back through the same (symmetric, orthogonal) transform
+            uint32_t acc[128];
+            float x[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 128; ++e) x[e] = (float)(int)acc[e] * __ldg(svb + e) * inv;
+#pragma unroll
+            for (int h = 1; h < 128; h <<= 1)
+#pragma unroll
+              for (int e = 0; e < 128; ++e)
+                if (!(e & h)) {
+                  const float u = x[e], w = x[e + h];
+                  x[e] = u + w;
+                  x[e + h] = u - w;
+                }
+            if (store) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                uint32_t hv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __half2 h2 = __floats2half2_rn(x[8 * q + 2 * e] * 0.08838834764831844055f,
+                                                       x[8 * q + 2 * e + 1] * 0.08838834764831844055f);
+                  hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                reinterpret_cast<uint4*>(orow)[q] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+              }
+            }
+          } else {
 #pragma unroll 1
           for (int c = 0; c < 8; ++c) {
             uint32_t acc[16];
@@ -400,6 +433,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               dst[0] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
               dst[1] = make_uint4(hv[4], hv[5], hv[6], hv[7]);
             }
+          }
           }
         }
       }

@@ -25,6 +25,7 @@ struct Prob {
   int n_tab;                    // table entries (each: cos, sin, alpha, beta)
   int rot;
   int p_mode;                   // ra_p_mode
+  int v_rot;                    // 1: Hadamard on V, undone on O (INT4 path)
   uint64_t signature;
 };
 

@@ -87,6 +87,34 @@ __device__ __forceinline__ void rope8(const Prob& P, const float4* __restrict__ 
   }
 }
 
+// Normalised 128-point Walsh-Hadamard transform of one row held by 16
+// consecutive lanes, 8 channels each (lane g: channels 8g .. 8g + 7): strides
+// 1, 2, 4 inside the lane, 8 .. 64 across lanes (lane bit h / 8); the pair
+// (k, k + h) becomes (a + b, a - b); then one multiply by fp32(1/sqrt(128)).
+// All 32 lanes of the warp must call it together.
+__device__ __forceinline__ void hadamard128(float (&z)[8], int g) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!(e & h)) {
+        const float a = z[e], b = z[e + h];
+        z[e] = __fadd_rn(a, b);
+        z[e + h] = __fsub_rn(a, b);
+      }
+#pragma unroll
+  for (int hl = 1; hl < 16; hl <<= 1) {
+    const bool upper = (g & hl) != 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, z[e], hl);
+      z[e] = upper ? __fsub_rn(other, z[e]) : __fadd_rn(z[e], other);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) z[e] = __fmul_rn(z[e], kRsqrt128);
+}
+
 __device__ __forceinline__ float block_max_128(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -152,32 +180,8 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
     }
   }
   if (ROT == RA_ROT_FULL) {
-    // normalised 128-point Walsh-Hadamard transform of every row, strides
-    // 1, 2, 4 inside a thread's 8 channels, 8 .. 64 across the 16 lanes that
-    // hold the row (lane bit h / 8); pair (k, k + h) -> (a + b, a - b)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-      for (int h = 1; h < 8; h <<= 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (!(e & h)) {
-            const float a = z[i][e], b = z[i][e + h];
-            z[i][e] = __fadd_rn(a, b);
-            z[i][e + h] = __fsub_rn(a, b);
-          }
-#pragma unroll
-      for (int hl = 1; hl < 16; hl <<= 1) {
-        const bool upper = (g & hl) != 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float other = __shfl_xor_sync(0xffffffffu, z[i][e], hl);
-          z[i][e] = upper ? __fsub_rn(other, z[i][e]) : __fadd_rn(z[i][e], other);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) z[i][e] = __fmul_rn(z[i][e], kRsqrt128);
-    }
+    for (int i = 0; i < 8; ++i) hadamard128(z[i], g);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i)
@@ -207,11 +211,20 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
   float m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int i = 0; i < 32; ++i) {
+  // rows past N count as zero rows; every lane runs every iteration, so the
+  // Hadamard's shuffles always see the whole warp
+  const int rows = min(256, P.N - chunk * 256);
+  const int iters = P.v_rot ? 32 : (rows + 7) / 8;
+  for (int i = 0; i < iters; ++i) {
     const int n = chunk * 256 + r0 + 8 * i;
-    if (n >= P.N) break;
     float f[8];
-    h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
+    if (n < P.N) {
+      h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+    }
+    if (P.v_rot) hadamard128(f, g);
 #pragma unroll
     for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
   }
@@ -251,6 +264,7 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = 0.0f;
     }
+    if (P.v_rot) hadamard128(f, g);
 #pragma unroll
     for (int e = 0; e < 8; ++e) codes[r0 + 8 * i][8 * g + e] = (int8_t)int4_code(f[e], s[e]);
   }

@@ -54,6 +54,7 @@ class Config:
     d: int = D_HEAD
     theta: float = 10000.0
     p_mode: str = "range"    # P quantisation: "range" (the method) | "symmetric"
+    v_rot: int = 0           # 1: Hadamard on V inside the INT4 path (undone on O)
 
     @property
     def N(self) -> int:

@@ -43,7 +43,7 @@ class _Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("n_text", ctypes.c_int), ("split", ctypes.c_int * 3),
-                ("theta", ctypes.c_double), ("rot", ctypes.c_int)]
+                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("v_rot", ctypes.c_int)]
 
 
 _lib = None
@@ -71,6 +71,7 @@ def problem(cfg, rot: Optional[str] = None) -> _Problem:
     p.split = (ctypes.c_int * 3)(*cfg.split)
     p.theta = float(cfg.theta)
     p.rot = ROT[rot if rot is not None else cfg.rot]
+    p.v_rot = int(getattr(cfg, "v_rot", 0))
     return p
 
 

@@ -43,7 +43,8 @@ typedef struct {
     int n_text;           /* text tokens appended after the video tokens */
     int split[3];         /* RoPE segment sizes (frame, height, width) */
     double theta;         /* RoPE base */
-    int rot;              /* 0 = no rotation, 1 = Interleaved, 2 = Half */
+    int rot;              /* 0 = no rotation, 1 = Interleaved, 2 = Half, 3 = Full */
+    int v_rot;            /* 1: Hadamard on V (INT4 path), undone on O */
 } orc_problem;
 
 enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2, ORC_ROT_FULL = 3 };
@@ -121,6 +122,39 @@ static void rope_row(const orc_problem *p, int n, const f16 *x, float *y)
  *                 (a, b) -> ((a+b)/sqrt2, (a-b)/sqrt2).
  * READING: rotation after RoPE (either order leaves QK^T unchanged); H2 is
  * the default block (free-parameter ledger). */
+/* Normalised Walsh-Hadamard transform z = y H / sqrt(d), H in Sylvester
+ * order (READING for the unspecified "Full" rotation and for the Hadamard the
+ * pages fuse into V), as the fast transform in fp32: for h = 1, 2, ..., d/2
+ * every pair (k, k + h) with k & h == 0 becomes (a + b, a - b); then one
+ * multiply by fp32(1/sqrt(d)).  y is overwritten. */
+static void hadamard_fp32(float *y, float *z, int d)
+{
+    for (int h = 1; h < d; h <<= 1)
+        for (int i = 0; i < d; i += 2 * h)
+            for (int k = i; k < i + h; ++k) {
+                float a = y[k], b = y[k + h];
+                y[k] = a + b;
+                y[k + h] = a - b;
+            }
+    const float r = (float)(1.0 / sqrt((double)(d)));
+    for (int c = 0; c < d; ++c) z[c] = y[c] * r;
+}
+
+/* The same transform in float64 (for undoing the V Hadamard on O: H is
+ * symmetric and orthogonal, so H^T = H). */
+static void hadamard_f64(double *y, int d)
+{
+    for (int w = 1; w < d; w *= 2)
+        for (int i = 0; i < d; i += 2 * w)
+            for (int k = i; k < i + w; ++k) {
+                double u = y[k], t = y[k + w];
+                y[k] = u + t;
+                y[k + w] = u - t;
+            }
+    const double r = 1.0 / sqrt((double)d);
+    for (int c = 0; c < d; ++c) y[c] *= r;
+}
+
 void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
 {
     if (p->rot == ORC_ROT_INTERLEAVED) {
@@ -147,22 +181,8 @@ void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
         memcpy(z, y, sizeof(float) * p->d);
         return;
     }
-    if (p->rot == ORC_ROT_FULL) {
-        /* "Full" rotation (the dense comparison of Figs. 4-5; READING: the
-         * normalised Walsh-Hadamard matrix H/sqrt(d), Sylvester order, as the
-         * fast transform: for h = 1, 2, ..., d/2 every pair (k, k + h) with
-         * k & h == 0 becomes (a + b, a - b) in fp32; then one multiply by
-         * fp32(1/sqrt(d)). */
-        int d = p->d;
-        for (int h = 1; h < d; h <<= 1)
-            for (int i = 0; i < d; i += 2 * h)
-                for (int k = i; k < i + h; ++k) {
-                    float a = y[k], b = y[k + h];
-                    y[k] = a + b;
-                    y[k + h] = a - b;
-                }
-        const float r = (float)(1.0 / sqrt((double)p->d));
-        for (int c = 0; c < d; ++c) z[c] = y[c] * r;
+    if (p->rot == ORC_ROT_FULL) {   /* the dense comparison of Figs. 4-5 */
+        hadamard_fp32(y, z, p->d);
         return;
     }
     const float r = (float)M_SQRT1_2;
@@ -232,7 +252,8 @@ void orc_quantize_qk_head(const orc_problem *p, const f16 *x, int8_t *codes, flo
 
 /* V of one head: one symmetric INT4 scale per channel over all N tokens
  * (amax_c / 7), codes in [-7, 7], and the per-64-token-block column sums of
- * the codes used by the zero-point correction.  No transform is applied to V:
+ * the codes used by the zero-point correction.  By default no transform is
+ * applied to V (v_rot = 0):
  * the paper's Hadamard on V is fused offline into the model weights.
  * codes: [N_pad][d]; sv: [d]; colsum: [N_pad/64][d].
  * READING: the pages fix no granularity for V; per-channel over the whole
@@ -240,10 +261,19 @@ void orc_quantize_qk_head(const orc_problem *p, const f16 *x, int8_t *codes, flo
 void orc_quantize_v_head(const orc_problem *p, const f16 *v, int8_t *codes, float *sv, int32_t *colsum)
 {
     int N = orc_seq_len(p), Np = orc_seq_pad(p), d = p->d;
+    /* V as fp32; with v_rot every row times H / sqrt(d) first (the stand-in
+     * for the Hadamard the pages fuse into V offline) */
+    float *vf = (float *)malloc(sizeof(float) * (size_t)N * d);
+    for (int n = 0; n < N; ++n) {
+        float y[512];
+        for (int c = 0; c < d; ++c) y[c] = (float)v[(size_t)n * d + c];
+        if (p->v_rot) hadamard_fp32(y, vf + (size_t)n * d, d);
+        else memcpy(vf + (size_t)n * d, y, sizeof(float) * d);
+    }
     for (int c = 0; c < d; ++c) {
         float amax = 0.0f;
         for (int n = 0; n < N; ++n) {
-            float a = fabsf((float)v[(size_t)n * d + c]);
+            float a = fabsf(vf[(size_t)n * d + c]);
             if (a > amax) amax = a;
         }
         sv[c] = amax / 7.0f;
@@ -252,10 +282,11 @@ void orc_quantize_v_head(const orc_problem *p, const f16 *v, int8_t *codes, floa
     memset(colsum, 0, sizeof(int32_t) * (size_t)(Np / QK_BLOCK) * d);
     for (int n = 0; n < N; ++n)
         for (int c = 0; c < d; ++c) {
-            int8_t q = int4_code((float)v[(size_t)n * d + c], sv[c]);
+            int8_t q = int4_code(vf[(size_t)n * d + c], sv[c]);
             codes[(size_t)n * d + c] = q;
             colsum[(size_t)(n / QK_BLOCK) * d + c] += q;
         }
+    free(vf);
 }
 
 /* Range-optimised P code: P in [0,1] -> rne(15 P) - 8 in [-8, 7]
@@ -357,8 +388,11 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
         l = l * alpha + L;
         m = m_new;
     }
+    double orow[512];
+    for (int c = 0; c < d; ++c) orow[c] = acc[c] * (double)sv[c] / l;
+    if (p->v_rot) hadamard_f64(orow, d);   /* O = O' H^T undoes V' = V H */
     for (int c = 0; c < d; ++c) {
-        double val = acc[c] * (double)sv[c] / l;
+        double val = orow[c];
         if (o64) o64[c] = val;
         if (o) o[c] = (f16)val;
     }

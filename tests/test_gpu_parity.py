@@ -85,6 +85,11 @@ SMALL = {
     "multi_tile": synth.Config("multi_tile", 1, 2, 4, 16, 20, 0, (44, 42, 42), "interleaved", "lognormal1.5", 15),
     # the Full (128-point Walsh-Hadamard) rotation, ragged, with text tokens
     "full_rot": synth.Config("full_rot", 1, 2, 3, 8, 10, 9, (44, 42, 42), "full", "lognormal1.5", 17),
+    # the Hadamard on V (undone on O), ragged with text tokens, and on Full rotation
+    "vrot_ragged": synth.Config("vrot_ragged", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 18,
+                                v_rot=1),
+    "vrot_full_sym": synth.Config("vrot_full_sym", 1, 2, 4, 8, 8, 0, (16, 56, 56), "full", "lognormal1.5", 19,
+                                  p_mode="symmetric", v_rot=1),
     # the symmetric P map (RA_P_SYMMETRIC) on a half-rotation and a ragged case
     "half_sym": synth.CONFIGS["half"].replace(name="half_sym", p_mode="symmetric"),
     "ragged_sym": synth.Config("ragged_sym", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 16,

@@ -24,7 +24,9 @@ MUTANTS = {
     "v_scale_per_tensor": ("sv[c] = amax / 7.0f;", "sv[c] = (amax > sv[0] ? amax : sv[0]) / 7.0f;"),
     "softmax_scale": ("(float)(1.0 / sqrt((double)d))", "(float)(1.0 / (double)d)"),
     "normaliser_exact_p": ("Li += code + zp;", "Li += 15;"),
-    "hadamard_sign": ("                    y[k + h] = a - b;", "                    y[k + h] = b - a;"),
+    "v_hadamard_not_undone": ("if (p->v_rot) hadamard_f64(orow, d);", "if (0) hadamard_f64(orow, d);"),
+    "v_hadamard_f64_sign": ("                y[k + w] = u - t;", "                y[k + w] = t - u;"),
+    "hadamard_sign": ("                y[k + h] = a - b;", "                y[k + h] = b - a;"),
     "hadamard_skips_stride_1": ("for (int h = 1; h < d; h <<= 1)", "for (int h = 2; h < d; h <<= 1)"),
     "p_sym_scale_8": ("nearbyintf(7.0f * P)", "nearbyintf(8.0f * P)"),
     "sym_keeps_zero_point": ("const int zp = quant_p == 2 ? 0 : 8;", "const int zp = 8;"),

@@ -370,6 +370,41 @@ def test_symmetric_p_single_tile_and_error_bound(oracle_mod):
     assert not np.array_equal(o_range, o_sym)
 
 
+def test_v_hadamard_quantiser_and_inverse(oracle_mod):
+    """v_rot = 1: V is quantised as V H / sqrt(128) (scipy's Hadamard, float64,
+    to fp32 rounding; codes within half a step of it) and the output row is
+    taken back through H: exact-P attention on the rotated V equals attention
+    on the dequantised rotated V times H, and both paths approximate
+    unquantised attention."""
+    from scipy.linalg import hadamard
+    H = hadamard(128).astype(np.float64) / math.sqrt(128)
+    cfg = small_cfg(F=2, Hh=6, W=10, n_text=7, rot="half", v_rot=1)        # N = 127
+    rng = np.random.default_rng(21)
+    q = (rng.standard_normal((cfg.N, 128)) * 0.8).astype(np.float16)
+    k = (rng.standard_normal((cfg.N, 128)) * 0.8).astype(np.float16)
+    v = rng.standard_normal((cfg.N, 128)).astype(np.float16)
+    v[:, 3] *= 8                                         # an outlier channel
+    vr = v.astype(np.float64) @ H
+    vc, sv, colsum = oracle_mod.quantize_v_head(cfg, v)
+    assert np.allclose(sv, np.abs(vr).max(axis=0) / 7, rtol=2e-6)
+    deq = vc[:cfg.N].astype(np.float64) * sv.astype(np.float64)
+    assert np.all(np.abs(deq - vr) <= sv.astype(np.float64) / 2 * (1 + 1e-5) + 1e-6)
+    qz = oracle_mod.quantize_head(cfg, q, k, v)
+    _, o_exactp = oracle_mod.attention_rows(cfg, qz, quant_p=False, want64=True)
+    S, s = dequant_logits(cfg, qz)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    ref = ((p / p.sum(axis=1, keepdims=True)) @ deq) @ H.T
+    assert np.allclose(o_exactp, ref, rtol=1e-6, atol=1e-7)   # fp32 logits in the oracle
+    exact = oracle_mod.exact_attention_rows(cfg, q, k, v)
+    _, o_rot = oracle_mod.attention_rows(cfg, qz, want64=True)
+    qz0 = oracle_mod.quantize_head(cfg.replace(v_rot=0), q, k, v)
+    _, o_plain = oracle_mod.attention_rows(cfg.replace(v_rot=0), qz0, want64=True)
+    # both approximate unquantised attention (INT4 Q, K, P and V on random
+    # data); without the inverse transform the cosine would be near 0
+    assert cos(o_rot, exact) > 0.95 and cos(o_plain, exact) > 0.95
+    assert not np.allclose(o_rot, o_plain, rtol=1e-9, atol=1e-9)
+
+
 def test_uniform_logits_give_the_mean(oracle_mod):
     """All keys equal -> P = 1 -> code 7 -> O = mean of the dequantised V."""
     cfg = small_cfg(F=3, Hh=8, W=8, rot="none")                        # N = 192
