@@ -47,12 +47,17 @@ typedef enum {
     RA_ROT_NONE = 0,            /* RoPE only */
     RA_ROT_INTERLEAVED = 1,     /* H2 on adjacent dims, merged into RoPE (Fig. 3) */
     RA_ROT_HALF = 2,            /* H2 on (i, i + d_s/2) in each segment (Fig. 3) */
-    RA_ROT_FULL = 3             /* dense rotation over all of head_dim after RoPE: the
+    RA_ROT_FULL = 3,            /* dense rotation over all of head_dim after RoPE: the
                                  * normalised 128-point Walsh-Hadamard transform (the
                                  * "Full" rotation the pages compare against, Figs. 4-5;
                                  * the matrix is not given there).  Computed as the fast
                                  * transform in fp32, strides 1, 2, ..., 64, then one
                                  * multiply by fp32(1/sqrt(128)). */
+    RA_ROT_BLOCKS_INTERLEAVED = 4, /* caller's 2x2 orthogonal block per adjacent pair
+                                 * (learned rotations, Sec. 4.1 / Fig. 6), merged into
+                                 * RoPE per (position, pair) like the Interleaved H2 */
+    RA_ROT_BLOCKS_HALF = 5      /* caller's 2x2 orthogonal block per (i, i + d_s/2)
+                                 * pair, applied after RoPE like the Half H2 */
 } ra_rot_mode;
 
 /* Quantisation of P = exp(s - m) in [0, 1] for the P.V product.
@@ -85,6 +90,12 @@ typedef struct {
                                  * quantising it and every output row by its transpose
                                  * (a stand-in for the Hadamard the pages fuse into V
                                  * offline: review page summary); 0: V as given */
+    const double *blocks;       /* host, d/2 x 4: block p = {r00, r01, r10, r11}, row
+                                 * major, rows orthonormal to 1e-6; needed for the
+                                 * BLOCKS modes (NULL otherwise).  Pair p of segment s
+                                 * is p = o_s / 2 + j (dims o_s + 2j, o_s + 2j + 1 for
+                                 * INTERLEAVED; o_s + j, o_s + j + d_s/2 for HALF);
+                                 * (z_a, z_b) = R (y_a, y_b). */
 } ra_problem;
 
 /* Quantised Q, K, V as produced by ra_rotate_quantize_qkv (device memory).

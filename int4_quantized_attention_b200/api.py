@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(PKG, "librotate_attn.so")
 
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_WORKSPACE, RA_ERR_CUDA, \
     RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(7)
-ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3}
+ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3, "blocks_interleaved": 4, "blocks_half": 5}
 P_MODE = {"range": 0, "symmetric": 1}       # ra_p_mode
 
 
@@ -32,7 +32,7 @@ class Problem(ctypes.Structure):
                 ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("n_text", ctypes.c_int), ("split", ctypes.c_int * 3),
                 ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("p_mode", ctypes.c_int),
-                ("v_rot", ctypes.c_int)]
+                ("v_rot", ctypes.c_int), ("blocks", ctypes.c_void_p)]
 
 
 class Qkv4(ctypes.Structure):
@@ -106,6 +106,11 @@ def problem(cfg, rot: Optional[str] = None) -> Problem:
     p.rot = ROT[rot if rot is not None else cfg.rot]
     p.p_mode = P_MODE[getattr(cfg, "p_mode", "range")]
     p.v_rot = int(getattr(cfg, "v_rot", 0))
+    blocks = getattr(cfg, "blocks", None)
+    if blocks is not None:
+        arr = (ctypes.c_double * len(blocks))(*blocks)
+        p._keep = arr                      # the array lives as long as the struct
+        p.blocks = ctypes.cast(arr, ctypes.c_void_p)
     return p
 
 

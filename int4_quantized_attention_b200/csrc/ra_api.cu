@@ -61,8 +61,19 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     sum += p->split[s];
   }
   if (sum != p->d) return fail(RA_ERR_INVALID_ARG, "RoPE split sums to %d, head_dim is %d", sum, p->d);
-  if (p->rot != RA_ROT_NONE && p->rot != RA_ROT_INTERLEAVED && p->rot != RA_ROT_HALF && p->rot != RA_ROT_FULL)
+  if (p->rot < RA_ROT_NONE || p->rot > RA_ROT_BLOCKS_HALF)
     return fail(RA_ERR_INVALID_ARG, "rotation mode %d unknown", p->rot);
+  const bool blocks = p->rot == RA_ROT_BLOCKS_INTERLEAVED || p->rot == RA_ROT_BLOCKS_HALF;
+  if (blocks) {
+    if (p->blocks == nullptr) return fail(RA_ERR_INVALID_ARG, "rotation mode %d needs the pair blocks", p->rot);
+    for (int q = 0; q < p->d / 2; ++q) {
+      const double* r = p->blocks + 4 * q;
+      const double e0 = r[0] * r[0] + r[1] * r[1] - 1.0, e1 = r[2] * r[2] + r[3] * r[3] - 1.0;
+      const double e2 = r[0] * r[2] + r[1] * r[3];
+      if (!(std::fabs(e0) < 1e-6 && std::fabs(e1) < 1e-6 && std::fabs(e2) < 1e-6))
+        return fail(RA_ERR_INVALID_ARG, "pair block %d is not orthogonal", q);
+    }
+  }
   if (!(p->theta > 0.0) || !std::isfinite(p->theta)) return fail(RA_ERR_INVALID_ARG, "RoPE base must be > 0");
   if (p->p_mode != RA_P_RANGE_OPTIMIZED && p->p_mode != RA_P_SYMMETRIC)
     return fail(RA_ERR_INVALID_ARG, "P quantisation mode %d unknown", p->p_mode);
@@ -95,10 +106,12 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
       toff += npos[s] * (p->split[s] / 2);
     }
     P.n_tab = toff;
+    P.n_tab_all = toff + p->d / 2;
     uint64_t h = fnv1a(&p->B, sizeof(int) * 7);
     h = fnv1a(p->split, sizeof(p->split), h);
     h = fnv1a(&p->theta, sizeof(double), h);
     h = fnv1a(&p->rot, sizeof(int), h);
+    if (blocks) h = fnv1a(p->blocks, sizeof(double) * 4 * (size_t)(p->d / 2), h);
     P.signature = h | 1ull;   // never 0, so a zeroed workspace never matches
   }
   return RA_OK;
@@ -108,6 +121,7 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
 // per (segment, position, pair), a = pos * theta^(-2j/d_s), each computed in
 // float64 and rounded once to fp32.
 void build_tables(const ra_problem* p, const ra::Prob& P, float* out) {
+  const bool blocks_mode = p->rot == RA_ROT_BLOCKS_INTERLEAVED || p->rot == RA_ROT_BLOCKS_HALF;
   for (int s = 0; s < 3; ++s) {
     const int half = p->split[s] / 2;
     for (int pos = 0; pos < P.npos[s]; ++pos)
@@ -116,12 +130,23 @@ void build_tables(const ra_problem* p, const ra::Prob& P, float* out) {
         const double a = (double)pos * w;
         const double ca = std::cos(a), sa = std::sin(a);
         float* e = out + 4 * ((size_t)P.tab_off[s] + (size_t)pos * half + j);
-        e[0] = (float)ca;
-        e[1] = (float)sa;
-        e[2] = (float)((ca + sa) * M_SQRT1_2);
-        e[3] = (float)((ca - sa) * M_SQRT1_2);
+        if (p->rot == RA_ROT_BLOCKS_INTERLEAVED) {   // R times the RoPE rotation, per (pos, pair)
+          const double* r = p->blocks + 4 * (P.off[s] / 2 + j);
+          e[0] = (float)(r[0] * ca + r[1] * sa);
+          e[1] = (float)(r[1] * ca - r[0] * sa);
+          e[2] = (float)(r[2] * ca + r[3] * sa);
+          e[3] = (float)(r[3] * ca - r[2] * sa);
+        } else {
+          e[0] = (float)ca;
+          e[1] = (float)sa;
+          e[2] = (float)((ca + sa) * M_SQRT1_2);
+          e[3] = (float)((ca - sa) * M_SQRT1_2);
+        }
       }
   }
+  // pair blocks, rounded to fp32 (used by BLOCKS_HALF), zero otherwise
+  for (int q = 0; q < p->d / 2; ++q)
+    for (int k = 0; k < 4; ++k) out[4 * ((size_t)P.n_tab + q) + k] = blocks_mode ? (float)p->blocks[4 * q + k] : 0.0f;
 }
 
 struct QkvLayout {
@@ -230,15 +255,15 @@ size_t ra_workspace_bytes(const ra_problem* p, int with_fp16_path) {
 size_t ra_tables_floats(const ra_problem* p) {
   ra::Prob P;
   if (derive(p, &P) != RA_OK) return 0;
-  return 4 * (size_t)P.n_tab;
+  return 4 * (size_t)P.n_tab_all;
 }
 
 ra_status ra_build_tables_host(const ra_problem* p, float* out, size_t n_floats) {
   ra::Prob P;
   ra_status st = derive(p, &P);
   if (st != RA_OK) return st;
-  if (out == nullptr || n_floats < 4 * (size_t)P.n_tab)
-    return fail(RA_ERR_INVALID_ARG, "table buffer NULL or smaller than %zu floats", 4 * (size_t)P.n_tab);
+  if (out == nullptr || n_floats < 4 * (size_t)P.n_tab_all)
+    return fail(RA_ERR_INVALID_ARG, "table buffer NULL or smaller than %zu floats", 4 * (size_t)P.n_tab_all);
   build_tables(p, P, out);
   return RA_OK;
 }
@@ -250,7 +275,7 @@ ra_status ra_prepare(const ra_problem* p, void* ws, size_t ws_bytes, ra_stream s
   if ((st = check_ws(P, ws, ws_bytes, WsUse::prologue)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const ra::WsLayout L = ra::ws_layout(P);
-  std::vector<float> tab(4 * (size_t)P.n_tab);
+  std::vector<float> tab(4 * (size_t)P.n_tab_all);
   build_tables(p, P, tab.data());
   ra::WsHeader hdr{};
   hdr.signature = P.signature;

@@ -22,7 +22,9 @@ struct Prob {
   int split[3], off[3];         // segment sizes and first channel of each segment
   int npos[3];                  // positions per axis: F, Hh, W
   int tab_off[3];               // first table entry of each segment
-  int n_tab;                    // table entries (each: cos, sin, alpha, beta)
+  int n_tab;                    // RoPE table entries (each: cos, sin, alpha, beta, or for
+                                // BLOCKS_INTERLEAVED the merged m00, m01, m10, m11)
+  int n_tab_all;                // n_tab + d/2 pair-block entries (r00, r01, r10, r11)
   int rot;
   int p_mode;                   // ra_p_mode
   int v_rot;                    // 1: Hadamard on V, undone on O (INT4 path)
@@ -54,7 +56,7 @@ inline WsLayout ws_layout(const Prob& p) {
   WsLayout L;
   size_t o = align256(sizeof(WsHeader));
   L.tables = o;
-  o = align256(o + sizeof(float) * 4 * (size_t)p.n_tab);
+  o = align256(o + sizeof(float) * 4 * (size_t)p.n_tab_all);
   L.vamax = o;
   o = align256(o + sizeof(uint32_t) * (size_t)p.BH * D);
   L.pro_bytes = o;

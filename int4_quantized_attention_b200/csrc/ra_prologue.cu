@@ -66,8 +66,10 @@ __device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P,
 }
 
 // RoPE of the 4 adjacent pairs held by one thread (channels c0..c0+7 of
-// token n); with MERGED the coefficient is the Interleaved H2*Rot form.
-template <bool MERGED>
+// token n).  FORM 0: the RoPE rotation (cos, sin); FORM 1: the Interleaved
+// H2 * Rot (alpha, beta); FORM 2: a caller's block times Rot, merged on the
+// host (m00, m01, m10, m11).
+template <int FORM>
 __device__ __forceinline__ void rope8(const Prob& P, const float4* __restrict__ tab, const TokenPos& tp, int c0,
                                       const float (&x)[8], float (&y)[8]) {
 #pragma unroll
@@ -77,10 +79,13 @@ __device__ __forceinline__ void rope8(const Prob& P, const float4* __restrict__ 
     const int j = (c - P.off[s]) >> 1;
     const float4 t = __ldg(&tab[P.tab_off[s] + tp.p[s] * (P.split[s] >> 1) + j]);
     const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
-    if (MERGED) {   // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
+    if (FORM == 1) {          // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
       y[2 * pp] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
       y[2 * pp + 1] = __fsub_rn(__fmul_rn(t.w, x0), __fmul_rn(t.z, x1));
-    } else {        // y0 = c x0 - s x1, y1 = s x0 + c x1
+    } else if (FORM == 2) {   // z0 = m00 x0 + m01 x1, z1 = m10 x0 + m11 x1
+      y[2 * pp] = __fadd_rn(__fmul_rn(t.x, x0), __fmul_rn(t.y, x1));
+      y[2 * pp + 1] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
+    } else {                  // y0 = c x0 - s x1, y1 = s x0 + c x1
       y[2 * pp] = __fsub_rn(__fmul_rn(t.x, x0), __fmul_rn(t.y, x1));
       y[2 * pp + 1] = __fadd_rn(__fmul_rn(t.y, x0), __fmul_rn(t.x, x1));
     }
@@ -133,7 +138,8 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
                                                        float* __restrict__ sk, const float4* __restrict__ tab,
                                                        const WsHeader* __restrict__ hdr) {
   __shared__ float red[4];
-  __shared__ float ys[ROT == RA_ROT_HALF ? QK_BLOCK : 1][ROT == RA_ROT_HALF ? D + 4 : 1];
+  constexpr bool HALF_PAIRS = ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF;
+  __shared__ float ys[HALF_PAIRS ? QK_BLOCK : 1][HALF_PAIRS ? D + 4 : 1];
   if (!signature_ok(hdr, P, 0x100)) return;
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
@@ -156,9 +162,9 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
     float xf[8];
     h8_to_f(raw[i], xf);
     const TokenPos tp = token_pos(P, n < P.N ? n : 0);
-    rope8<ROT == RA_ROT_INTERLEAVED>(P, tab, tp, c0, xf, z[i]);
+    rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(P, tab, tp, c0, xf, z[i]);
   }
-  if (ROT == RA_ROT_HALF) {
+  if (HALF_PAIRS) {
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -170,12 +176,19 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
       const int s = segment_of(P, c);
       const int h = P.split[s] >> 1;
       const bool first = (c - P.off[s]) < h;
+      float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ROT == RA_ROT_BLOCKS_HALF)   // block of pair off_s / 2 + i, i = index in the first half
+        r4 = __ldg(&tab[P.n_tab + (P.off[s] >> 1) + (c - P.off[s]) - (first ? 0 : h)]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = r0 + 8 * i;
         const float a = first ? ys[r][c] : ys[r][c - h];
         const float b = first ? ys[r][c + h] : ys[r][c];
-        z[i][e] = first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
+        if (ROT == RA_ROT_BLOCKS_HALF)
+          z[i][e] = first ? __fadd_rn(__fmul_rn(r4.x, a), __fmul_rn(r4.y, b))
+                          : __fadd_rn(__fmul_rn(r4.z, a), __fmul_rn(r4.w, b));
+        else
+          z[i][e] = first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
       }
     }
   }
@@ -318,7 +331,7 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
       if (n < P.N) {
         float xf[8], y[8];
         h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)), xf);
-        rope8<false>(P, tab, token_pos(P, n), c0, xf, y);
+        rope8<0>(P, tab, token_pos(P, n), c0, xf, y);
         __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
@@ -368,6 +381,12 @@ cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, con
       qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
       break;
     case RA_ROT_FULL: qk_quant_kernel<RA_ROT_FULL><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    case RA_ROT_BLOCKS_INTERLEAVED:
+      qk_quant_kernel<RA_ROT_BLOCKS_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      break;
+    case RA_ROT_BLOCKS_HALF:
+      qk_quant_kernel<RA_ROT_BLOCKS_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      break;
     default: qk_quant_kernel<RA_ROT_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
   }
   cudaError_t e = cudaGetLastError();

@@ -55,6 +55,7 @@ class Config:
     theta: float = 10000.0
     p_mode: str = "range"    # P quantisation: "range" (the method) | "symmetric"
     v_rot: int = 0           # 1: Hadamard on V inside the INT4 path (undone on O)
+    blocks: Optional[tuple] = None   # rot "blocks_*": d/2 x (r00, r01, r10, r11), flattened
 
     @property
     def N(self) -> int:
@@ -78,6 +79,18 @@ CONFIGS = {
     "hunyuan": Config("hunyuan", 1, 24, 33, 45, 80, 256, (16, 56, 56), "half", "lognormal1.5", 104),
     "wan_flat": Config("wan_flat", 1, 40, 21, 45, 80, 0, (44, 42, 42), "interleaved", "const0.3", 105),
 }
+
+def random_pair_blocks(seed: int, d: int = D_HEAD) -> tuple:
+    """d/2 seeded 2x2 orthogonal blocks (a rotation or a reflection each),
+    flattened row-major: stand-ins for learned rotations."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for _ in range(d // 2):
+        t = rng.uniform(-np.pi, np.pi)
+        c, s = np.cos(t), np.sin(t)
+        out += [c, -s, s, c] if rng.random() < 0.5 else [c, s, s, -c]
+    return tuple(float(v) for v in out)
+
 
 def _channel_scales(cfg: Config, rng: np.random.Generator) -> np.ndarray:
     """Per-(head, channel) float32 scale shared by Q and K."""

@@ -17,7 +17,7 @@ import numpy as np
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "rotate_attn_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
-ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3}
+ROT = {"none": 0, "interleaved": 1, "half": 2, "full": 3, "blocks_interleaved": 4, "blocks_half": 5}
 
 
 def compile_oracle(src: str, out: str) -> None:
@@ -43,7 +43,8 @@ class _Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("F", ctypes.c_int), ("Hh", ctypes.c_int), ("W", ctypes.c_int),
                 ("n_text", ctypes.c_int), ("split", ctypes.c_int * 3),
-                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("v_rot", ctypes.c_int)]
+                ("theta", ctypes.c_double), ("rot", ctypes.c_int), ("v_rot", ctypes.c_int),
+                ("blocks", ctypes.c_void_p)]
 
 
 _lib = None
@@ -72,6 +73,11 @@ def problem(cfg, rot: Optional[str] = None) -> _Problem:
     p.theta = float(cfg.theta)
     p.rot = ROT[rot if rot is not None else cfg.rot]
     p.v_rot = int(getattr(cfg, "v_rot", 0))
+    blocks = getattr(cfg, "blocks", None)
+    if blocks is not None:
+        arr = (ctypes.c_double * len(blocks))(*blocks)
+        p._keep = arr                      # the array lives as long as the struct
+        p.blocks = ctypes.cast(arr, ctypes.c_void_p)
     return p
 
 

@@ -45,9 +45,11 @@ typedef struct {
     double theta;         /* RoPE base */
     int rot;              /* 0 = no rotation, 1 = Interleaved, 2 = Half, 3 = Full */
     int v_rot;            /* 1: Hadamard on V (INT4 path), undone on O */
+    const double *blocks; /* rot 4/5: d/2 caller 2x2 blocks {r00, r01, r10, r11} */
 } orc_problem;
 
-enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2, ORC_ROT_FULL = 3 };
+enum { ORC_ROT_NONE = 0, ORC_ROT_INTERLEAVED = 1, ORC_ROT_HALF = 2, ORC_ROT_FULL = 3,
+       ORC_ROT_BLOCKS_INTERLEAVED = 4, ORC_ROT_BLOCKS_HALF = 5 };
 enum { QK_BLOCK = 64, KV_TILE = 128 };
 
 int orc_seq_len(const orc_problem *p) { return p->F * p->Hh * p->W + p->n_text; }
@@ -157,6 +159,28 @@ static void hadamard_f64(double *y, int d)
 
 void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
 {
+    if (p->rot == ORC_ROT_BLOCKS_INTERLEAVED) {
+        /* caller's orthogonal block R_p on the adjacent pair p = o_s / 2 + j,
+         * merged with the RoPE rotation: M = R Rot(a) in float64, rounded once */
+        int pos[3];
+        orc_token_pos(p, n, pos);
+        int o = 0;
+        for (int s = 0; s < 3; ++s) {
+            for (int j = 0; j < p->split[s] / 2; ++j) {
+                double a = orc_rope_angle(p, s, pos[s], j);
+                double ca = cos(a), sa = sin(a);
+                const double *R = p->blocks + 4 * (o / 2 + j);
+                float m00 = (float)(R[0] * ca + R[1] * sa), m01 = (float)(R[1] * ca - R[0] * sa);
+                float m10 = (float)(R[2] * ca + R[3] * sa), m11 = (float)(R[3] * ca - R[2] * sa);
+                float x0 = (float)x[o + 2 * j], x1 = (float)x[o + 2 * j + 1];
+                float t0 = m00 * x0, t1 = m01 * x1, t2 = m10 * x0, t3 = m11 * x1;
+                z[o + 2 * j] = t0 + t1;
+                z[o + 2 * j + 1] = t2 + t3;
+            }
+            o += p->split[s];
+        }
+        return;
+    }
     if (p->rot == ORC_ROT_INTERLEAVED) {
         int pos[3];
         orc_token_pos(p, n, pos);
@@ -183,6 +207,24 @@ void orc_rotate_row(const orc_problem *p, int n, const f16 *x, float *z)
     }
     if (p->rot == ORC_ROT_FULL) {   /* the dense comparison of Figs. 4-5 */
         hadamard_fp32(y, z, p->d);
+        return;
+    }
+    if (p->rot == ORC_ROT_BLOCKS_HALF) {
+        /* caller's orthogonal block R_p on (o_s + i, o_s + i + d_s/2) after RoPE,
+         * p = o_s / 2 + i (learned rotations, Sec. 4.1); R rounded to fp32 */
+        int o = 0;
+        for (int s = 0; s < 3; ++s) {
+            int h = p->split[s] / 2;
+            for (int i = 0; i < h; ++i) {
+                const double *R = p->blocks + 4 * (o / 2 + i);
+                float r00 = (float)R[0], r01 = (float)R[1], r10 = (float)R[2], r11 = (float)R[3];
+                float ya = y[o + i], yb = y[o + i + h];
+                float t0 = r00 * ya, t1 = r01 * yb, t2 = r10 * ya, t3 = r11 * yb;
+                z[o + i] = t0 + t1;
+                z[o + i + h] = t2 + t3;
+            }
+            o += p->split[s];
+        }
         return;
     }
     const float r = (float)M_SQRT1_2;

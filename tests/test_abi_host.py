@@ -53,6 +53,11 @@ def test_validation_codes(lib):
     bad = prob()
     bad.p_mode = 2                                                           # unknown P map
     assert api.validate(bad) == api.RA_ERR_INVALID_ARG
+    blocks = synth.random_pair_blocks(1)
+    assert api.validate(prob(rot="blocks_half", blocks=blocks)) == api.RA_OK
+    assert api.validate(prob(rot="blocks_interleaved")) == api.RA_ERR_INVALID_ARG     # no blocks
+    skew = tuple(b * 1.01 for b in blocks)                                   # not orthogonal
+    assert api.validate(prob(rot="blocks_half", blocks=skew)) == api.RA_ERR_INVALID_ARG
     assert api.validate(prob(theta=0.0)) == api.RA_ERR_INVALID_ARG
     p = prob()
     p.rot = 7
@@ -121,4 +126,5 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
             got = tab[k + pos * half + j]
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (name, s, pos, j)
         k += npos[s] * half
-    assert k == len(tab)
+    assert k + 64 == len(tab)                 # then the 64 pair-block entries (zero here)
+    assert not tab[k:].any()

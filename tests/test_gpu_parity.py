@@ -90,6 +90,11 @@ SMALL = {
                                 v_rot=1),
     "vrot_full_sym": synth.Config("vrot_full_sym", 1, 2, 4, 8, 8, 0, (16, 56, 56), "full", "lognormal1.5", 19,
                                   p_mode="symmetric", v_rot=1),
+    # caller 2x2 pair blocks (learned-rotation stand-ins), merged into RoPE / after RoPE
+    "blocks_il": synth.Config("blocks_il", 1, 2, 3, 7, 9, 5, (44, 42, 42), "blocks_interleaved", "lognormal1.5", 20,
+                              blocks=synth.random_pair_blocks(40)),
+    "blocks_half": synth.Config("blocks_half", 1, 2, 2, 9, 10, 40, (16, 56, 56), "blocks_half", "lognormal1.5", 21,
+                                blocks=synth.random_pair_blocks(41)),
     # the symmetric P map (RA_P_SYMMETRIC) on a half-rotation and a ragged case
     "half_sym": synth.CONFIGS["half"].replace(name="half_sym", p_mode="symmetric"),
     "ragged_sym": synth.Config("ragged_sym", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 16,

@@ -24,6 +24,8 @@ MUTANTS = {
     "v_scale_per_tensor": ("sv[c] = amax / 7.0f;", "sv[c] = (amax > sv[0] ? amax : sv[0]) / 7.0f;"),
     "softmax_scale": ("(float)(1.0 / sqrt((double)d))", "(float)(1.0 / (double)d)"),
     "normaliser_exact_p": ("Li += code + zp;", "Li += 15;"),
+    "blocks_merge_sign": ("m01 = (float)(R[1] * ca - R[0] * sa)", "m01 = (float)(R[1] * ca + R[0] * sa)"),
+    "blocks_half_transposed": ("r10 = (float)R[2], r11 = (float)R[3];", "r10 = (float)R[1], r11 = (float)R[3];"),
     "v_hadamard_not_undone": ("if (p->v_rot) hadamard_f64(orow, d);", "if (0) hadamard_f64(orow, d);"),
     "v_hadamard_f64_sign": ("                y[k + w] = u - t;", "                y[k + w] = t - u;"),
     "hadamard_sign": ("                y[k + h] = a - b;", "                y[k + h] = b - a;"),

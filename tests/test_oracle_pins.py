@@ -232,6 +232,47 @@ def test_full_rotation_is_the_normalised_hadamard(oracle_mod):
     assert np.allclose(np.abs(zz), 1 / math.sqrt(128), rtol=1e-6)
 
 
+def _block_diag(blocks, split, mode):
+    """The d x d matrix (column-vector convention z = M y) of the pair blocks."""
+    M = np.zeros((128, 128))
+    o = 0
+    for seg in split:
+        h = seg // 2
+        for j in range(h):
+            p = o // 2 + j
+            r = np.array(blocks[4 * p:4 * p + 4]).reshape(2, 2)
+            a, b = (o + 2 * j, o + 2 * j + 1) if mode == "blocks_interleaved" else (o + j, o + j + h)
+            M[np.ix_([a, b], [a, b])] = r
+        o += seg
+    return M
+
+
+@pytest.mark.parametrize("mode", ["blocks_interleaved", "blocks_half"])
+@pytest.mark.parametrize("split", [(44, 42, 42), (16, 56, 56)])
+def test_learned_blocks_are_the_block_diagonal_matrix(oracle_mod, mode, split):
+    """Caller blocks: z = B (RoPE y) with B block-diagonal over the pairs of the
+    mode (numpy, float64) to fp32 rounding; QK^T and norms preserved; with the
+    exact H2 blocks the modes reproduce Interleaved / Half to fp32 rounding."""
+    blocks = synth.random_pair_blocks(31)
+    cfg = small_cfg(F=2, Hh=3, W=4, n_text=2, split=split, rot=mode, blocks=blocks)
+    rng = np.random.default_rng(4)
+    q = (rng.standard_normal((cfg.N, 128)) * 2).astype(np.float16)
+    k = (rng.standard_normal((cfg.N, 128)) * 2).astype(np.float16)
+    y = oracle_mod.rotate_head(cfg, q, rot="none").astype(np.float64)
+    yk = oracle_mod.rotate_head(cfg, k, rot="none").astype(np.float64)
+    z = oracle_mod.rotate_head(cfg, q).astype(np.float64)
+    zk = oracle_mod.rotate_head(cfg, k).astype(np.float64)
+    ref = y @ _block_diag(blocks, split, mode).T
+    assert np.max(np.abs(z - ref)) <= 2e-6 * np.max(np.abs(ref))
+    qk = y @ yk.T
+    assert np.max(np.abs(z @ zk.T - qk)) <= 1e-5 * np.max(np.abs(qk))
+    h2 = tuple([math.sqrt(0.5), math.sqrt(0.5), math.sqrt(0.5), -math.sqrt(0.5)] * 64)
+    std = "interleaved" if mode == "blocks_interleaved" else "half"
+    zh = oracle_mod.rotate_head(cfg.replace(blocks=h2), q).astype(np.float64)
+    zs = oracle_mod.rotate_head(cfg.replace(rot=std, blocks=None), q).astype(np.float64)
+    assert np.max(np.abs(zh - zs)) <= 2e-6 * np.max(np.abs(zs))
+
+
 # ---------------------------------------------------------------- quantisers
 
 @pytest.mark.parametrize("rot", ["interleaved", "half", "full"])
