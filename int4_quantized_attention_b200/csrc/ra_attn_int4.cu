@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         const bool dbg_tile = dbg_run && (qt0 + X) == a.dbg_qt;
         const int tail = P.N - (nt - 1) * TILE;   // valid keys in the last tile, 1..128
         float m = -INFINITY, l = 0.0f;
+        bool zbuf0 = false, zbuf1 = false;   // this warp's rows of P buffer 0 / 1 hold zeros
         float skn0 = __ldg(skb), skn1 = __ldg(skb + 1);
         for (int j = 0; j < nt; ++j) {
           const float sk0 = skn0, sk1 = skn1;
@@ -309,11 +310,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
 #pragma unroll
             for (int k = 16 * h; k < 16 * h + 16; k += 2) {   // 8 keys per pair of words: evens, then odds
               uint32_t wb[8];
+              const float ch = h ? c1 : c0;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 8; e += 2) {   // x = (s - MAGIC) c - m, w = rne(pscale 2^x): pairs
                 const int n = 4 * k + e;
-                const float x = fmaf(__int_as_float(s[n]) - MAGIC, h ? c1 : c0, negm);
-                wb[e] = __float_as_uint(fmaf(pscale, ex2(x), MAGIC));   // low byte = w
+                float x0, x1, w0, w1;
+                add2(x0, x1, __int_as_float(s[n]), __int_as_float(s[n + 1]), -MAGIC, -MAGIC);
+                fma2(x0, x1, x0, x1, ch, ch, negm, negm);
+                fma2(w0, w1, pscale, pscale, ex2(x0), ex2(x1), MAGIC, MAGIC);   // low byte = w
+                wb[e] = __float_as_uint(w0);
+                wb[e + 1] = __float_as_uint(w1);
               }
               const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
               const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
@@ -350,9 +356,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
             for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
             tmem_wait_st();
           }
-          // P buffer j % 2 is free again once P.V(j-2) has read it
-          if (j >= 2 && !(ok = wait_all(B_PV_DONE + 2 * X + (j & 1), ((j - 2) >> 1) & 1, 0x4103))) break;
-          {
+          // P buffer j % 2 is free: its last reader P.V(j-2) was issued before
+          // S(j) by the same thread, so the arrival of S(j) means it has landed.
+          // A warp whose rows are all zero and whose rows of the buffer already
+          // hold zeros leaves them as they are.
+          const bool all_zero = zero_half[0] && zero_half[1] && nvalid == TILE;
+          if (!(all_zero && ((j & 1) ? zbuf1 : zbuf0))) {
             uint8_t* prow = sm + Smem::P + (2 * X + (j & 1)) * 16384;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -360,6 +369,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
                   make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             fence_async_smem();
           }
+          if (j & 1) zbuf1 = all_zero; else zbuf0 = all_zero;
           l = fmaf(l, alpha, (float)L);
           if (dbg_tile && j == a.dbg_kv) {
 #pragma unroll
