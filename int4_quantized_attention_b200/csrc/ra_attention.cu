@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(f16::NUM_THREADS, 1)
         }
         const bool zero_half[2] = {__all_sync(0xffffffffu, mx0 - m < SKIP_BELOW) != 0,
                                    __all_sync(0xffffffffu, mx1 - m < SKIP_BELOW) != 0};
-        float lsum = 0.0f;
+        float lsum0 = 0.0f, lsum1 = 0.0f;   // row sum over even / odd keys
         uint32_t ph[64];   // P as fp16 pairs: ph[c] = keys 2c (low), 2c + 1
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -186,15 +186,16 @@ __global__ void __launch_bounds__(f16::NUM_THREADS, 1)
             continue;
           }
 #pragma unroll
-          for (int c = 32 * h; c < 32 * h + 32; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), cs, negm));
-            const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), cs, negm));
-            lsum += p0 + p1;
+          for (int c = 32 * h; c < 32 * h + 32; ++c) {   // pairs of keys on packed fp32 pairs
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]), cs, cs, negm, negm);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            add2(lsum0, lsum1, lsum0, lsum1, p0, p1);
             const __half2 h2 = __floats2half2_rn(p0, p1);
             ph[c] = *reinterpret_cast<const uint32_t*>(&h2);
           }
         }
-        l = fmaf(l, alpha, lsum);
+        l = fmaf(l, alpha, lsum0 + lsum1);
         tmem_st32(tS + 64, ph);
         tmem_st32(tS + 96, ph + 32);
         tmem_wait_st();
