@@ -120,24 +120,33 @@ __device__ __forceinline__ void hadamard128(float (&z)[8], int g) {
   for (int e = 0; e < 8; ++e) z[e] = __fmul_rn(z[e], kRsqrt128);
 }
 
-__device__ __forceinline__ float block_max_128(float v, float* red) {
+// Q/K prologue CTA: one 64-token block of one head, QK_THREADS threads; lane
+// g = t % 16 holds channels 8g .. 8g + 7 of rows t / 16 + QK_RSTEP i (four
+// rows a thread: 64 registers, half the SM's warp slots, against a quarter
+// with eight rows).
+constexpr int QK_THREADS = 256, QK_RSTEP = QK_THREADS / 16, QK_ROWS = QK_BLOCK / QK_RSTEP;
+
+__device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   __syncthreads();
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
-  return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float m = red[0];
+#pragma unroll
+  for (int w = 1; w < QK_THREADS / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
 }
 
-// One CTA = one 64-token block of Q or K of one head (128 threads).  Thread
-// t holds channels 8*(t%16) .. +7 of rows (t/16) + 8i, i = 0..7.
+// One CTA = one 64-token block of Q or K of one head (QK_THREADS threads).
+// Thread t holds channels 8*(t%16) .. +7 of rows (t/16) + QK_RSTEP i.
 template <int ROT>
-__global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __restrict__ q,
+__global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __half* __restrict__ q,
                                                        const __half* __restrict__ k, uint8_t* __restrict__ q4,
                                                        uint8_t* __restrict__ k4, float* __restrict__ sq,
                                                        float* __restrict__ sk, const float4* __restrict__ tab,
                                                        const WsHeader* __restrict__ hdr) {
-  __shared__ float red[4];
+  __shared__ float red[QK_THREADS / 32];
   constexpr bool HALF_PAIRS = ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF;
   __shared__ float ys[HALF_PAIRS ? QK_BLOCK : 1][HALF_PAIRS ? D + 4 : 1];
   if (!signature_ok(hdr, P, 0x100)) return;
@@ -145,20 +154,20 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
   const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
   uint8_t* out = (which ? k4 : q4) + (size_t)bh * P.N_pad * (D / 2);
   float* scale = (which ? sk : sq) + (size_t)bh * (P.N_pad / QK_BLOCK);
-  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;   // rows r0 + QK_RSTEP i
   const int c0 = 8 * g;
 
-  uint4 raw[8];
+  uint4 raw[QK_ROWS];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = blk * QK_BLOCK + r0 + 8 * i;
+  for (int i = 0; i < QK_ROWS; ++i) {
+    const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     raw[i] = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
   }
-  float z[8][8];
+  float z[QK_ROWS][8];
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = blk * QK_BLOCK + r0 + 8 * i;
+  for (int i = 0; i < QK_ROWS; ++i) {
+    const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     float xf[8];
     h8_to_f(raw[i], xf);
     const TokenPos tp = token_pos(P, n < P.N ? n : 0);
@@ -166,9 +175,9 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
   }
   if (HALF_PAIRS) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < QK_ROWS; ++i)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ys[r0 + 8 * i][c0 + e] = z[i][e];
+      for (int e = 0; e < 8; ++e) ys[r0 + QK_RSTEP * i][c0 + e] = z[i][e];
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
@@ -180,8 +189,8 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
       if (ROT == RA_ROT_BLOCKS_HALF)   // block of pair off_s / 2 + i, i = index in the first half
         r4 = __ldg(&tab[P.n_tab + (P.off[s] >> 1) + (c - P.off[s]) - (first ? 0 : h)]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = r0 + 8 * i;
+      for (int i = 0; i < QK_ROWS; ++i) {
+        const int r = r0 + QK_RSTEP * i;
         const float a = first ? ys[r][c] : ys[r][c - h];
         const float b = first ? ys[r][c + h] : ys[r][c];
         if (ROT == RA_ROT_BLOCKS_HALF)
@@ -194,17 +203,17 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(Prob P, const __half* __r
   }
   if (ROT == RA_ROT_FULL) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) hadamard128(z[i], g);
+    for (int i = 0; i < QK_ROWS; ++i) hadamard128(z[i], g);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < QK_ROWS; ++i)
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(z[i][e]));
-  amax = block_max_128(amax, red);
+  amax = block_max(amax, red);
   const float s = __fdiv_rn(amax, 7.0f);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = blk * QK_BLOCK + r0 + 8 * i;
+  for (int i = 0; i < QK_ROWS; ++i) {
+    const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     uint32_t packed = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) packed |= (uint32_t)(int4_code(z[i][e], s) & 0xF) << (4 * e);
@@ -376,18 +385,18 @@ cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, con
   uint32_t* vamax = reinterpret_cast<uint32_t*>(base + L.vamax);
   const dim3 gqk(p.N_pad / QK_BLOCK, p.BH, 2);
   switch (p.rot) {
-    case RA_ROT_NONE: qk_quant_kernel<RA_ROT_NONE><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    case RA_ROT_NONE: qk_quant_kernel<RA_ROT_NONE><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
     case RA_ROT_INTERLEAVED:
-      qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
       break;
-    case RA_ROT_FULL: qk_quant_kernel<RA_ROT_FULL><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    case RA_ROT_FULL: qk_quant_kernel<RA_ROT_FULL><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
     case RA_ROT_BLOCKS_INTERLEAVED:
-      qk_quant_kernel<RA_ROT_BLOCKS_INTERLEAVED><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      qk_quant_kernel<RA_ROT_BLOCKS_INTERLEAVED><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
       break;
     case RA_ROT_BLOCKS_HALF:
-      qk_quant_kernel<RA_ROT_BLOCKS_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      qk_quant_kernel<RA_ROT_BLOCKS_HALF><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
       break;
-    default: qk_quant_kernel<RA_ROT_HALF><<<gqk, 128, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    default: qk_quant_kernel<RA_ROT_HALF><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
