@@ -231,3 +231,26 @@ def test_full_size_sampled(oracle_mod, dev, name):
         g = o[b, h][rows].astype(np.float64)
         assert cosine(g, out64) >= COS_MIN, (bh, cosine(g, out64))
         assert np.abs(g - out64).max() <= MAXABS_INT4 * np.abs(v[b, h].astype(np.float64)).max()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_fp16_full_size_sampled(oracle_mod, dev, name):
+    """The FP16 path at full size in the benchmark's launch configuration:
+    sampled rows of the first, the last and a middle head against float64
+    attention on the fp16-rounded RoPE inputs (always the ragged last row)."""
+    cfg = synth.CONFIGS[name]
+    q, k, v = synth.make_qkv(cfg)
+    ra = api.RotateAttention(cfg, dev, fp16_path=True)
+    o = ra.fp16_attention(*(to_dev(t, dev) for t in (q, k, v)))
+    ra.check()
+    o = o.cpu().numpy()
+    BH, N = cfg.B * cfg.H, cfg.N
+    rng = np.random.default_rng(98)
+    for bh in (0, BH // 2, BH - 1):
+        b, h = divmod(bh, cfg.H)
+        rows = np.unique(np.concatenate([rng.choice(N, 24, replace=False), [0, N - 1]])).astype(np.int64)
+        ref = oracle_mod.fp16_attention_rows(cfg, q[b, h], k[b, h], v[b, h], rows=rows)
+        g = o[b, h][rows].astype(np.float64)
+        assert cosine(g, ref) >= COS_MIN, (bh, cosine(g, ref))
+        assert np.abs(g - ref).max() <= MAXABS_FP16 * np.abs(v[b, h].astype(np.float64)).max()
