@@ -77,6 +77,27 @@ def test_sizes(lib):
         min_qkv = 3 * BH * Np * 64 + 2 * BH * (Np // 64) * 4 + BH * 128 * 4 + BH * (Np // 64) * 128 * 4
         assert api.qkv4_bytes(p) >= min_qkv
         assert api.workspace_bytes(p, True) >= api.workspace_bytes(p, False) + 3 * BH * Np * 128 * 2
+        # the INT4 path holds the INT8 operand images of Q, K and V^T
+        assert api.workspace_bytes(p, False) >= 3 * BH * Np * 128
+
+
+def test_each_call_checks_its_own_workspace_size(lib):
+    """The prologue needs only header, tables and V amax; the INT4 attention
+    also needs the operand images: a workspace between the two sizes serves
+    the first and is refused (RA_ERR_WORKSPACE) by the second, before any
+    launch."""
+    cfg = synth.CONFIGS["tiny"]
+    p = api.problem(cfg)
+    full = api.workspace_bytes(p, False)
+    Np, BH = api.seq_pad(p), cfg.B * cfg.H
+    mid = full - 3 * BH * Np * 128                      # room for everything but the images
+    q = api.Qkv4()
+    assert lib.ra_qkv4_bind(ctypes.byref(p), 256, 1 << 30, ctypes.byref(q)) == api.RA_OK
+    st = lib.ra_int4_attention_fwd(ctypes.byref(p), ctypes.byref(q), 256, 256, mid, None)
+    assert st == api.RA_ERR_WORKSPACE
+    assert b"needs" in lib.ra_last_error_detail()
+    st = lib.ra_fp16_attention_fwd(ctypes.byref(p), 256, 256, 256, 256, 256, full, None)
+    assert st == api.RA_ERR_WORKSPACE                   # the FP16 path needs its images too
 
 
 def test_calls_reject_bad_arguments_without_a_gpu(lib):
