@@ -43,9 +43,9 @@
 // symmetric P map instead: w = rne(7 * 2^(x - m)) = code), fed as an
 // unsigned 8-bit operand: the tensor core then sums (code + 8) * v, which is
 // sum code * v + 8 * colsum(v) -- the zero-point correction, bit-identical.
-// The int32 P.V accumulator stays in TMEM across tiles; the rescale is an
-// integer multiply by round(2^31 * exp(m_old - m_new)) (exp(...) is exactly
-// 1 for every other row).  The normaliser l is the running sum of w.
+// The int32 P.V accumulator stays in TMEM across tiles; the rescale rounds
+// acc * exp2(m_old - m_new) back to an integer (rows whose max did not move
+// keep theirs).  The normaliser l is the running sum of w.
 //
 // INT4 codes are expanded to 16*code (the nibble placed in the high half of
 // the byte), so S comes out as 256*S and P.V as 16*P.V, exactly; both factors
@@ -102,6 +102,13 @@ enum : int {
 __device__ __forceinline__ void widen16(const uint4 u, uint4& a, uint4& b) {
   a = make_uint4((u.x << 4) & 0xF0F0F0F0u, u.x & 0xF0F0F0F0u, (u.y << 4) & 0xF0F0F0F0u, u.y & 0xF0F0F0F0u);
   b = make_uint4((u.z << 4) & 0xF0F0F0F0u, u.z & 0xF0F0F0F0u, (u.w << 4) & 0xF0F0F0F0u, u.w & 0xF0F0F0F0u);
+}
+
+// All 128 columns of this warp's 32 lanes in one load.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+               : "r"(taddr));
 }
 
 // P word k (0..31) holds, in byte b, key 8 (k / 2) + 2 b + (k % 2).  Byte mask
@@ -256,8 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           if (!(ok = wait_all(B_S_FULL + X, j & 1, 0x4102))) break;
           tc_fence_after();
           uint32_t s[128];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+          tmem_ld128(tS, s);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
@@ -337,25 +343,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               pw[k] &= keep;
             }
           }
-          // rows whose max moved: acc *= alpha after P.V(j-1) has landed (it
-          // was issued a whole tile ago) and before P.V(j) adds to it
-          if (__any_sync(0xffffffffu, moved)) {
-            if (!(ok = wait_all(B_PV_DONE + 2 * X + ((j - 1) & 1), ((j - 1) >> 1) & 1, 0x4104))) break;
-            tc_fence_after();
-            // acc * alpha = (2 acc * round(2^31 alpha)) >> 32, |acc| < 2^28
-            const int aq = __float2int_rn(fminf(alpha * 2147483648.0f, 2147483520.0f));
-            uint32_t acc[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
-            tmem_wait_ld();
-            if (moved) {
-#pragma unroll
-              for (int e = 0; e < 128; ++e) acc[e] = (uint32_t)__mulhi((int)acc[e] * 2, aq);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
-            tmem_wait_st();
-          }
           // P buffer j % 2 is free: its last reader P.V(j-2) was issued before
           // S(j) by the same thread, so the arrival of S(j) means it has landed.
           // A warp whose rows are all zero and whose rows of the buffer already
@@ -368,6 +355,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               *reinterpret_cast<uint4*>(prow + sw128_off(row, c)) =
                   make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             fence_async_smem();
+          }
+          // rows whose max moved: acc *= alpha after P.V(j-1) has landed (it
+          // was issued a whole tile ago) and before P.V(j) adds to it.  The
+          // product is taken in fp32 and rounded to an integer by adding
+          // 1.5 * 2^23, whose last mantissa bit is worth 1.  |acc| <= 112 l
+          // plus one unit per earlier rescale, so while l < 2^15 both acc and
+          // the product lie below 2^22 and the result is the nearest integer
+          // to acc * alpha.  Larger rows round acc * alpha / 64 (|acc| < 2^28)
+          // and scale it back: at most 64 units off, under 1e-4 s_V in O as
+          // l >= 2^15 there.  A warp with no such row takes the short loop.
+          if (__any_sync(0xffffffffu, moved)) {
+            if (!(ok = wait_all(B_PV_DONE + 2 * X + ((j - 1) & 1), ((j - 1) >> 1) & 1, 0x4104))) break;
+            tc_fence_after();
+            const bool big = l >= 32768.0f;
+            const bool any_big = __any_sync(0xffffffffu, moved && big);
+            uint32_t acc[128];
+            tmem_ld128(tO, acc);
+            tmem_wait_ld();
+            if (moved) {
+              if (!any_big) {
+#pragma unroll
+                for (int e = 0; e < 128; e += 2) {
+                  float r0, r1;
+                  fma2(r0, r1, __int2float_rn((int)acc[e]), __int2float_rn((int)acc[e + 1]), alpha, alpha, MAGIC,
+                       MAGIC);
+                  acc[e] = __float_as_uint(r0) - (uint32_t)MAGIC_BITS;
+                  acc[e + 1] = __float_as_uint(r1) - (uint32_t)MAGIC_BITS;
+                }
+              } else {
+                const float sc = big ? alpha * 0.015625f : alpha;
+                const uint32_t mult = big ? 64u : 1u, add = 0u - (uint32_t)MAGIC_BITS * mult;
+#pragma unroll
+                for (int e = 0; e < 128; e += 2) {
+                  float r0, r1;
+                  fma2(r0, r1, __int2float_rn((int)acc[e]), __int2float_rn((int)acc[e + 1]), sc, sc, MAGIC, MAGIC);
+                  acc[e] = __float_as_uint(r0) * mult + add;
+                  acc[e + 1] = __float_as_uint(r1) * mult + add;
+                }
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, acc + 32 * c);
+            tmem_wait_st();
           }
           if (j & 1) zbuf1 = all_zero; else zbuf0 = all_zero;
           l = fmaf(l, alpha, (float)L);

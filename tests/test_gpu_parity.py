@@ -99,6 +99,9 @@ SMALL = {
     "half_sym": synth.CONFIGS["half"].replace(name="half_sym", p_mode="symmetric"),
     "ragged_sym": synth.Config("ragged_sym", 1, 2, 3, 7, 9, 5, (44, 42, 42), "interleaved", "lognormal1", 16,
                                p_mode="symmetric"),
+    # flat logits over N = 4*24*50 + 7 = 4807 keys: the normaliser passes 2^15
+    # early, so late rescales take the large-row path of the accumulator
+    "flat_long": synth.Config("flat_long", 1, 2, 4, 24, 50, 7, (44, 42, 42), "interleaved", "const0.3", 22),
 }
 
 
