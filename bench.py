@@ -248,11 +248,15 @@ def our_arm(args, cfg, rank, world):
     ms_f16 = event_time(lambda: ra.fp16_attention(qd, kd, vd, out), max(2, args.steps // 3), stream)
     ra.check()
 
-    # end to end through the public API with host buffers
+    # end to end with host buffers: ra_int4_attention_host pipelines the copies
+    # over chunks of heads on the copy engines while the kernels run
     qh, kh, vh = (torch.from_numpy(t).pin_memory() for t in (q, k, v))
     oh = torch.empty(out.shape, dtype=torch.float16).pin_memory()
 
     def e2e_step():
+        ra.forward_host(qh, kh, vh, oh, heads_per_chunk=args.chunk_heads)
+
+    def e2e_serial():
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
@@ -261,6 +265,7 @@ def our_arm(args, cfg, rank, world):
 
     e2e_step()
     ms_e2e = event_time(e2e_step, max(2, args.steps // 2), stream)
+    ms_e2e_serial = event_time(e2e_serial, 2, stream)
     ra.check()
     ms_e2e = max_over_ranks(ms_e2e, dev)
 
@@ -307,7 +312,10 @@ def our_arm(args, cfg, rank, world):
                       "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TF/s (the call is timed alone)",
                       "int4_step_speedup": ms_f16 / ms_step},
         "e2e": {"value": aggregate_tops(world, ops, ms_e2e), "unit": "TOPS", "ms_per_step": ms_e2e,
-                "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2},
+                "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2,
+                "api": "ra_int4_attention_host (pinned host q, k, v, o; copies overlapped over head chunks)",
+                "heads_per_chunk": args.chunk_heads or -(-BH // 8),
+                "serial_ms_per_step": ms_e2e_serial},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample",
@@ -363,6 +371,8 @@ def main():
     ap.add_argument("--v-rot", action="store_true", help="Hadamard on V inside the INT4 path (undone on O)")
     ap.add_argument("--p-mode", default="range", choices=["range", "symmetric"],
                     help="P quantisation of the INT4 path (range-optimised: the method)")
+    ap.add_argument("--chunk-heads", type=int, default=0,
+                    help="heads per chunk of the host-buffer pipeline (0: the library's default, B*H/8)")
     ap.add_argument("--only-step", action="store_true",
                     help="run only the warm-up and timed INT4 steps (for profiler captures)")
     args = ap.parse_args()

@@ -9,11 +9,13 @@
  *
  * Conventions for every entry point:
  *   - Tensors are DEVICE pointers, 16-byte aligned, row-major and contiguous.
- *     fp16 tensors are [B][H][N][d] with d = 128.
+ *     fp16 tensors are [B][H][N][d] with d = 128.  (ra_int4_attention_host
+ *     alone takes host q, k, v, o.)
  *   - The caller owns all memory.  The library allocates and frees nothing on
  *     any call; it only reads and writes the buffers it is given.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
- *     stream) and returns without synchronising, except ra_check_device_error.
+ *     stream) and returns without synchronising, except ra_check_device_error
+ *     and ra_int4_attention_host.
  *   - Errors are status codes; nothing throws or aborts across the ABI.
  *     Argument errors are found on the host before any launch and nothing is
  *     enqueued then.  ra_last_error_detail() gives a one-line reason for the
@@ -146,7 +148,11 @@ size_t ra_workspace_bytes(const ra_problem *p, int with_fp16_path);
  * with cudaMemcpyAsync on `stream`, clears the error word and records the
  * problem's signature.  Call once per (problem, workspace) before the other
  * calls; they check the signature on the device and report
- * RA_ERR_WORKSPACE through ra_check_device_error when it does not match. */
+ * RA_ERR_WORKSPACE through ra_check_device_error when it does not match.
+ * The signature covers what the tables depend on (d, grid, text tokens,
+ * split, theta, rotation, pair blocks), not B or H: a workspace prepared
+ * once serves problems that differ only in batch or head count, as long as
+ * it is large enough for them. */
 ra_status ra_prepare(const ra_problem *p, void *workspace, size_t workspace_bytes, ra_stream stream);
 
 /* Fused prologue: 3D RoPE and the RoPE-aware rotation of Q and K, per
@@ -175,6 +181,33 @@ ra_status ra_int4_attention_fwd(const ra_problem *p, const ra_qkv4 *in, void *o,
  * with with_fp16_path != 0. */
 ra_status ra_fp16_attention_fwd(const ra_problem *p, const void *q, const void *k, const void *v,
                                 void *o, void *workspace, size_t workspace_bytes, ra_stream stream);
+
+/* ---- INT4 forward on host buffers ------------------------------------- */
+
+/* Device bytes of the staging buffer ra_int4_attention_host needs (0 if the
+ * problem or heads_per_chunk is invalid). */
+size_t ra_host_staging_bytes(const ra_problem *p, int heads_per_chunk);
+
+/* The whole INT4 path (ra_rotate_quantize_qkv, then ra_int4_attention_fwd)
+ * from HOST q, k, v to HOST o, all fp16 [B][H][N][128], with the transfers
+ * overlapped with the kernels.  The B*H heads, flattened, are processed in
+ * chunks of consecutive heads, each chunk as a problem of its own with B = 1
+ * (every step of the path is independent per head, so the results are
+ * bit-identical to the device-buffer calls).  heads_per_chunk > 0: chunks of
+ * that many heads; 0: chunks of 1, 2, 3, ... heads growing to about B*H/8,
+ * so that the kernels start after a one-head copy.  While chunk c is computed on `stream`, the inputs
+ * of chunk c+1 are copied in and the output of chunk c-1 is copied out on
+ * two streams the call creates and destroys.  The copies overlap only if the
+ * host buffers are page-locked (cudaHostAlloc / cudaHostRegister); pageable
+ * buffers give the same result without the overlap.
+ * staging: device memory owned by the caller, 256-byte aligned, at least
+ * ra_host_staging_bytes(p, heads_per_chunk) bytes: two slots of q, k, v, o
+ * for the largest chunk plus the quantised tensors and workspace of one.  The
+ * call blocks until o is written and the device error words are checked,
+ * so it returns any status ra_check_device_error can.  The staging buffer
+ * must not be used by other work while the call runs. */
+ra_status ra_int4_attention_host(const ra_problem *p, const void *q, const void *k, const void *v, void *o,
+                                 int heads_per_chunk, void *staging, size_t staging_bytes, ra_stream stream);
 
 /* Synchronises `stream`, reads and clears the workspace's error word.
  * Returns RA_OK, RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS or

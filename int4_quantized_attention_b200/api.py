@@ -59,6 +59,8 @@ _SIGNATURES = {
     "ra_int4_attention_fwd": (ctypes.c_int, [_P, ctypes.POINTER(Qkv4), _V, _V, _SZ, _V]),
     "ra_fp16_attention_fwd": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _SZ, _V]),
     "ra_check_device_error": (ctypes.c_int, [_V, _V]),
+    "ra_host_staging_bytes": (_SZ, [_P, ctypes.c_int]),
+    "ra_int4_attention_host": (ctypes.c_int, [_P, _V, _V, _V, _V, ctypes.c_int, _V, _SZ, _V]),
     "ra_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ra_last_error_detail": (ctypes.c_char_p, []),
     "ra_tables_floats": (_SZ, [_P]),
@@ -175,6 +177,18 @@ def fp16_attention_fwd(p: Problem, q, k, v, o, workspace, stream=None) -> None:
                                        workspace.numel(), _stream(stream)))
 
 
+def host_staging_bytes(p: Problem, heads_per_chunk: int = 0) -> int:
+    return lib().ra_host_staging_bytes(ctypes.byref(p), heads_per_chunk)
+
+
+def int4_attention_host(p: Problem, q, k, v, o, staging, heads_per_chunk: int = 0, stream=None) -> None:
+    """The INT4 path from host q, k, v to host o (CPU tensors, page-locked for
+    overlap); blocks until o is written."""
+    _check("ra_int4_attention_host",
+           lib().ra_int4_attention_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), heads_per_chunk,
+                                        _ptr(staging), staging.numel(), _stream(stream)))
+
+
 def rotate_quantize_qkv_noalloc(p: Problem, q, k, v, out: Qkv4, stream=None) -> None:
     """The prologue with its scratch in the library's fixed device array."""
     _check("ra_rotate_quantize_qkv_noalloc",
@@ -260,6 +274,17 @@ class RotateAttention:
         if path == "fp16":
             return self.fp16_attention(q, k, v, out)
         raise ValueError(path)
+
+    def forward_host(self, q, k, v, out, heads_per_chunk: int = 0):
+        """INT4 path on host tensors (q, k, v, out on the CPU, page-locked for
+        overlap): copies, kernels and copies back pipelined over head chunks
+        by the library.  Returns once out is written."""
+        import torch
+        need = host_staging_bytes(self.p, heads_per_chunk)
+        if getattr(self, "_staging", None) is None or self._staging.numel() < need:
+            self._staging = torch.empty((need,), dtype=torch.uint8, device=self.device)
+        int4_attention_host(self.p, q, k, v, out, self._staging, heads_per_chunk)
+        return out
 
     def check(self) -> None:
         check_device_error(self.workspace)

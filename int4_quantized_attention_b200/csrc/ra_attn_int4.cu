@@ -16,7 +16,7 @@
 //                      3-stage ring
 //       warps 9, 10    MMA issuers, one thread per query tile (warp 9 also
 //                      owns the TMEM allocation)
-//       warp 11        writes the constant bf16 operand at start-up
+//       warp 11        idle after set-up
 // The packed INT4 inputs are expanded once per call, by expand_kernel, into
 // INT8 operand images laid out exactly as the MMAs read them from SMEM, so
 // the attention kernel itself only copies tiles.
@@ -34,10 +34,9 @@
 // its own softmax thread, after P.V(j-1) has landed (issued a whole tile
 // earlier) and before it releases W(j).
 //
-// S_X(j) starts as 1.5 * 2^23 in every accumulator (one bf16 MMA with a
-// constant operand), so after the integer MMAs add 256 S the accumulator bits
-// are exactly the float 1.5 * 2^23 + 256 S: the softmax takes its row max and
-// its exponent arguments on the raw bits, with no integer-to-float step.
+// S_X(j) is the int32 256 S of the four integer MMAs (the first one starts
+// the accumulator).  The softmax takes the row max on the integers and
+// converts to fp32 (exact: |256 S| < 2^24) only what it exponentiates.
 //
 // The P operand is w = rne(15 * 2^(x - m)) = code + 8 in [0, 15] (with the
 // symmetric P map instead: w = rne(7 * 2^(x - m)) = code), fed as an
@@ -74,19 +73,20 @@ static_assert(256 * SOFTMAX_REGS + 128 * ISSUE_REGS <= NUM_THREADS * LAUNCH_REGS
 
 constexpr uint32_t IDESC_QK = make_idesc(2, 1, 1, 128, 128);   // s32 += s8 x s8
 constexpr uint32_t IDESC_PV = make_idesc(2, 0, 1, 128, 128);   // s32 += u8 x s8
-constexpr uint32_t IDESC_INIT = make_idesc(1, 1, 1, 128, 128);  // f32 = bf16 x bf16
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float SQRT_D = 11.313708498984761f;
 constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
 constexpr int MAGIC_BITS = 0x4B400000;
-constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6), still exact through MAGIC
+constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6)
+
+// max of three int32 (two compares)
+__device__ __forceinline__ int imax3(int a, int b, int c) { return max(max(a, b), c); }
 
 struct Smem {
   static constexpr uint32_t QA = 0, QB = 16384;   // INT8 Q operand tiles
   static constexpr uint32_t OP = 32768;           // 3 x 32 KB: INT8 K (+0), V^T (+16 KB)
   static constexpr uint32_t P = 131072;           // [tile][j % 2] 16 KB u8 P operands, laid out like Q
-  static constexpr uint32_t CT = 196608;          // 4 KB: bf16 operand that sets S to 1.5 * 2^23
-  static constexpr uint32_t BAR = 200704;
+  static constexpr uint32_t BAR = 196608;
   static constexpr uint32_t BYTES = BAR + 512;
 };
 
@@ -207,17 +207,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
     tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
-  if (warp == 11) {
-    // bf16 2048 in columns 0..2 of every row, zero elsewhere: used as both
-    // operands, A B^T = 3 * 2048^2 = 1.5 * 2^23 in every accumulator, whose
-    // bits 0x4B400000 the integer S MMAs then add 256 S to
-    uint32_t* ct = reinterpret_cast<uint32_t*>(sm + Smem::CT);
-    for (int i = lane; i < 1024; i += 32) {
-      const int w = i & 3;   // row i / 4 holds K elements 0..7 in bytes 16 r .. 16 r + 15
-      ct[i] = i >= 512 ? 0u : (w == 0 ? 0x45004500u : (w == 1 ? 0x00004500u : 0u));
-    }
-    fence_async_smem();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -271,29 +260,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           const int nvalid = (j == nt - 1) ? tail : TILE;
           if (dbg_tile && j == a.dbg_kv) {   // S = (256 S) >> 8, exactly
 #pragma unroll
-            for (int n = 0; n < 128; ++n) a.dbg_s[row * TILE + n] = n < nvalid ? ((int)(s[n] - MAGIC_BITS) >> 8) : 0;
+            for (int n = 0; n < 128; ++n) a.dbg_s[row * TILE + n] = n < nvalid ? ((int)s[n] >> 8) : 0;
           }
           if (nvalid < TILE) {
 #pragma unroll
             for (int n = 0; n < 128; ++n)
-              if (n >= nvalid) s[n] = (uint32_t)(MAGIC_BITS + S_PAD);
+              if (n >= nvalid) s[n] = (uint32_t)S_PAD;
           }
           const float c0 = __fmul_rn(kq, sk0), c1 = __fmul_rn(kq, sk1);
-          // row max: the accumulators hold the bits of the floats 1.5*2^23 +
-          // 256 S, exact and ordered like S
-          float mh[8];
+          // row max of the int32 256 S of each 64-key half, then as floats
+          // (exact: |256 S| < 2^24)
+          int mh[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            mh[c] = fmax3(__int_as_float(s[16 * c]), __int_as_float(s[16 * c + 1]), __int_as_float(s[16 * c + 2]));
+            mh[c] = imax3((int)s[16 * c], (int)s[16 * c + 1], (int)s[16 * c + 2]);
 #pragma unroll
-            for (int n = 3; n < 15; n += 2)
-              mh[c] = fmax3(mh[c], __int_as_float(s[16 * c + n]), __int_as_float(s[16 * c + n + 1]));
-            mh[c] = fmaxf(mh[c], __int_as_float(s[16 * c + 15]));
+            for (int n = 3; n < 15; n += 2) mh[c] = imax3(mh[c], (int)s[16 * c + n], (int)s[16 * c + n + 1]);
+            mh[c] = max(mh[c], (int)s[16 * c + 15]);
           }
-          const float mx0 = fmaxf(fmax3(mh[0], mh[1], mh[2]), mh[3]);
-          const float mx1 = fmaxf(fmax3(mh[4], mh[5], mh[6]), mh[7]);
-          float tmax = __fmul_rn(mx0 - MAGIC, c0);
-          if (nvalid > 64) tmax = fmaxf(tmax, __fmul_rn(mx1 - MAGIC, c1));
+          const float mx0 = __int2float_rn(max(imax3(mh[0], mh[1], mh[2]), mh[3]));
+          const float mx1 = __int2float_rn(max(imax3(mh[4], mh[5], mh[6]), mh[7]));
+          float tmax = __fmul_rn(mx0, c0);
+          if (nvalid > 64) tmax = fmaxf(tmax, __fmul_rn(mx1, c1));
           const float m_new = fmaxf(m, tmax);
           const bool moved = j > 0 && m_new > m;
           const float alpha = moved ? ex2(m - m_new) : 1.0f;
@@ -302,8 +290,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
           // 64-key half whose largest x is below -5 holds only zero codes.
           // Skip its exponentials when that is so for every row of the warp.
-          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0 - MAGIC, c0, negm) < skip_below) != 0,
-                                     __all_sync(0xffffffffu, fmaf(mx1 - MAGIC, c1, negm) < skip_below) != 0};
+          const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0, c0, negm) < skip_below) != 0,
+                                     __all_sync(0xffffffffu, fmaf(mx1, c1, negm) < skip_below) != 0};
           uint32_t L = 0;
           uint32_t pw[32];
 #pragma unroll
@@ -318,11 +306,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               uint32_t wb[8];
               const float ch = h ? c1 : c0;
 #pragma unroll
-              for (int e = 0; e < 8; e += 2) {   // x = (s - MAGIC) c - m, w = rne(pscale 2^x): pairs
+              for (int e = 0; e < 8; e += 2) {   // x = 256 S c - m, w = rne(pscale 2^x): pairs
                 const int n = 4 * k + e;
                 float x0, x1, w0, w1;
-                add2(x0, x1, __int_as_float(s[n]), __int_as_float(s[n + 1]), -MAGIC, -MAGIC);
-                fma2(x0, x1, x0, x1, ch, ch, negm, negm);
+                fma2(x0, x1, __int2float_rn((int)s[n]), __int2float_rn((int)s[n + 1]), ch, ch, negm, negm);
                 fma2(w0, w1, pscale, pscale, ex2(x0), ex2(x1), MAGIC, MAGIC);   // low byte = w
                 wb[e] = __float_as_uint(w0);
                 wb[e + 1] = __float_as_uint(w1);
@@ -521,17 +508,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       const uint32_t qa = smem_u32(sm + (X ? Smem::QB : Smem::QA));
       const uint32_t pbase = smem_u32(sm + Smem::P + 2 * X * 16384);
       const uint32_t op = smem_u32(sm + Smem::OP);
-      const uint64_t dc = plain_desc(smem_u32(sm + Smem::CT));
       const uint32_t tS = tbase + X * 128, tO = tbase + 256 + X * 128;
       auto wait = [&](int b, uint32_t parity, uint32_t site) {
         return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
       };
-      auto issue_S = [&](int j) {   // S_X(j): set to 1.5 * 2^23, then += 256 Q_X K(j)^T
+      auto issue_S = [&](int j) {   // S_X(j) = 256 Q_X K(j)^T
         const uint32_t kt = op + (j % OP_STAGES) * 32768;
-        umma_f16(tS, dc, dc, IDESC_INIT, 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, 1);
+          umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, kk > 0);
         umma_commit(&bar[B_S_FULL + X]);
       };
       bool ok = wait(B_QFULL, 0, 0x4301) && wait(B_OP_FULL, 0, 0x4302);

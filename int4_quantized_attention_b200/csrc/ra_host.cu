@@ -1,0 +1,205 @@
+// ra_host.cu -- the INT4 forward from and to host memory, with the copies
+// overlapped with the kernels.
+//
+// Heads are independent in every step of the path (Q/K blocks, V channel
+// scales and the attention all live inside one (b, h)), so the flattened
+// B*H heads are cut into chunks of consecutive heads, each a problem of its
+// own with B = 1.  Three streams form a pipeline over the chunks:
+//
+//   copy-in stream : q, k, v of chunk c, host -> slot c % 2
+//   caller's stream: prologue + INT4 attention of chunk c (slot c % 2)
+//   copy-out stream: o of chunk c, slot c % 2 -> host
+//
+// so that the host->device copy of chunk c+1 and the device->host copy of
+// chunk c-1 run on the copy engines while chunk c is computed.  Events order
+// the reuse of the two slots.  The call blocks until o is written.
+#include <algorithm>
+#include <cstdio>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "ra_internal.h"
+
+namespace {
+
+constexpr int kDefaultChunks = 8;   // chunks of the largest size when the caller passes 0
+
+struct HostPlan {
+  std::vector<int> heads;     // heads of every chunk, in order
+  int BH, per;                // flattened heads; the largest chunk
+  ra_problem chunk;           // B = 1, H = per (sizes the regions below)
+  size_t head_bytes;          // one head of one fp16 tensor: N * 128 * 2
+  size_t ws, qkv4, slot;      // region sizes (256-aligned)
+  size_t off_qkv4, off_slots, total;
+};
+
+// Chunk sizes.  Given heads_per_chunk > 0: equal chunks (the last one takes
+// the remainder).  Given 0: chunks of about B*H/8 heads, reached by a ramp
+// 1, 2, 3, ... so that the first kernels wait only for a one-head copy (the
+// copy of a head takes about 3/4 of its compute, so each chunk's copy-in
+// hides behind the previous chunk's kernels when sizes grow by at most 4/3).
+void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
+  out.clear();
+  if (heads_per_chunk > 0) {
+    for (int h0 = 0; h0 < BH; h0 += heads_per_chunk) out.push_back(std::min(heads_per_chunk, BH - h0));
+    return;
+  }
+  const int per = (BH + kDefaultChunks - 1) / kDefaultChunks;
+  int done = 0, next = 1;
+  while (done < BH) {
+    const int c = std::min(std::min(next, per), BH - done);
+    out.push_back(c);
+    done += c;
+    next = std::max(next + 1, (4 * c) / 3);
+  }
+}
+
+ra_status plan(const ra_problem* p, int heads_per_chunk, HostPlan* hp) {
+  ra::Prob P;
+  ra_status st = ra::derive_problem(p, &P);
+  if (st != RA_OK) return st;
+  if (heads_per_chunk < 0) {
+    ra::set_error_detail("heads_per_chunk must be >= 0 (0: the library's default)");
+    return RA_ERR_INVALID_ARG;
+  }
+  HostPlan& h = *hp;
+  h.BH = P.BH;
+  chunk_sizes(P.BH, heads_per_chunk, h.heads);
+  h.per = *std::max_element(h.heads.begin(), h.heads.end());
+  h.chunk = *p;
+  h.chunk.B = 1;
+  h.chunk.H = h.per;
+  h.head_bytes = (size_t)P.N * ra::D * 2;
+  h.ws = ra::align256(ra_workspace_bytes(&h.chunk, 0));
+  h.qkv4 = ra::align256(ra_qkv4_bytes(&h.chunk));
+  h.slot = ra::align256(4 * h.per * h.head_bytes);    // q, k, v, o of one chunk
+  h.off_qkv4 = h.ws;
+  h.off_slots = h.off_qkv4 + h.qkv4;
+  h.total = h.off_slots + 2 * h.slot;
+  return RA_OK;
+}
+
+ra_status cuda_err(cudaError_t e, const char* what) {
+  char buf[200];
+  snprintf(buf, sizeof(buf), "%s: %s", what, cudaGetErrorString(e));
+  cudaGetLastError();
+  ra::set_error_detail(buf);
+  return RA_ERR_CUDA;
+}
+
+// Streams and events of one call, released on every path out of it.
+struct Pipeline {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t loaded[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr}, stored[2] = {nullptr, nullptr};
+  ~Pipeline() {
+    for (int i = 0; i < 2; ++i) {
+      if (loaded[i]) cudaEventDestroy(loaded[i]);
+      if (computed[i]) cudaEventDestroy(computed[i]);
+      if (stored[i]) cudaEventDestroy(stored[i]);
+    }
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+  cudaError_t create() {
+    cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&loaded[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&stored[i], cudaEventDisableTiming);
+    }
+    return e;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t ra_host_staging_bytes(const ra_problem* p, int heads_per_chunk) {
+  HostPlan h;
+  return plan(p, heads_per_chunk, &h) == RA_OK ? h.total : 0;
+}
+
+ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void* k, const void* v, void* o,
+                                 int heads_per_chunk, void* staging, size_t staging_bytes, ra_stream stream) {
+  HostPlan h;
+  ra_status st = plan(p, heads_per_chunk, &h);
+  if (st != RA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) {
+    ra::set_error_detail("host q, k, v or o is NULL");
+    return RA_ERR_INVALID_ARG;
+  }
+  if (staging == nullptr || (reinterpret_cast<uintptr_t>(staging) & 255u)) {
+    ra::set_error_detail("staging buffer NULL or not 256-byte aligned");
+    return RA_ERR_INVALID_ARG;
+  }
+  if (staging_bytes < h.total) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "staging buffer has %zu bytes, needs %zu", staging_bytes, h.total);
+    ra::set_error_detail(buf);
+    return RA_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(staging);
+  void* ws = base;
+
+  // Tables and signature (synchronises `stream`); the signature does not
+  // cover B or H, so this workspace serves every chunk.
+  if ((st = ra_prepare(&h.chunk, ws, h.ws, stream)) != RA_OK) return st;
+
+  Pipeline pl;
+  cudaError_t e = pl.create();
+  if (e != cudaSuccess) return cuda_err(e, "stream/event creation");
+
+  const char* qh = static_cast<const char*>(q);
+  const char* kh = static_cast<const char*>(k);
+  const char* vh = static_cast<const char*>(v);
+  char* oh = static_cast<char*>(o);
+  size_t off = 0;   // first byte of the chunk in every host tensor
+  for (size_t c = 0; c < h.heads.size(); ++c) {
+    const int sl = (int)(c & 1);
+    ra_problem cp = h.chunk;
+    cp.H = h.heads[c];
+    ra_qkv4 qkv;
+    if ((st = ra_qkv4_bind(&cp, base + h.off_qkv4, h.qkv4, &qkv)) != RA_OK) break;
+    const size_t n = (size_t)cp.H * h.head_bytes;
+    char* slot = base + h.off_slots + sl * h.slot;
+    char *qd = slot, *kd = slot + n, *vd = slot + 2 * n, *od = slot + 3 * n;
+
+    // copy-in: the slot's inputs are free once chunk c-2 has been computed
+    if (c >= 2 && (e = cudaStreamWaitEvent(pl.in, pl.computed[sl], 0)) != cudaSuccess) break;
+    if ((e = cudaMemcpyAsync(qd, qh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
+    if ((e = cudaMemcpyAsync(kd, kh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
+    if ((e = cudaMemcpyAsync(vd, vh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
+    if ((e = cudaEventRecord(pl.loaded[sl], pl.in)) != cudaSuccess) break;
+
+    // compute: inputs loaded, and the slot's output read back (chunk c-2)
+    if ((e = cudaStreamWaitEvent(s, pl.loaded[sl], 0)) != cudaSuccess) break;
+    if (c >= 2 && (e = cudaStreamWaitEvent(s, pl.stored[sl], 0)) != cudaSuccess) break;
+    if ((st = ra_rotate_quantize_qkv(&cp, qd, kd, vd, &qkv, ws, h.ws, stream)) != RA_OK) break;
+    if ((st = ra_int4_attention_fwd(&cp, &qkv, od, ws, h.ws, stream)) != RA_OK) break;
+    if ((e = cudaEventRecord(pl.computed[sl], s)) != cudaSuccess) break;
+
+    // copy-out
+    if ((e = cudaStreamWaitEvent(pl.out, pl.computed[sl], 0)) != cudaSuccess) break;
+    if ((e = cudaMemcpyAsync(oh + off, od, n, cudaMemcpyDeviceToHost, pl.out)) != cudaSuccess) break;
+    if ((e = cudaEventRecord(pl.stored[sl], pl.out)) != cudaSuccess) break;
+    off += n;
+  }
+  // Join both copy streams into the caller's stream, then wait for all of it,
+  // also on an error path (nothing may still use the staging buffer on return).
+  cudaError_t j = cudaEventRecord(pl.loaded[0], pl.in);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.loaded[0], 0);
+  if (j == cudaSuccess) j = cudaEventRecord(pl.stored[0], pl.out);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.stored[0], 0);
+  cudaError_t w = cudaStreamSynchronize(s);
+  if (st != RA_OK) return st;
+  if (e != cudaSuccess) return cuda_err(e, "pipeline enqueue");
+  if (j != cudaSuccess) return cuda_err(j, "pipeline join");
+  if (w != cudaSuccess) return cuda_err(w, "pipeline synchronize");
+  return ra_check_device_error(ws, stream);
+}
+
+}  // extern "C"

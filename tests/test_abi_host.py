@@ -128,6 +128,39 @@ def test_calls_reject_bad_arguments_without_a_gpu(lib):
         assert api.status_string(s)
 
 
+def test_host_entry_plan_and_argument_checks(lib):
+    """ra_int4_attention_host: the staging size covers two chunk slots of
+    q, k, v, o plus one chunk's quantised tensors and workspace; bad
+    arguments are refused before any CUDA call."""
+    cfg = synth.CONFIGS["wan"]
+    p = api.problem(cfg)
+    head = cfg.N * 128 * 2
+    for per in (1, 5, 7, 40):
+        chunk = api.problem(cfg.replace(H=per))
+        need = api.host_staging_bytes(p, per)
+        assert need >= 2 * 4 * per * head + api.workspace_bytes(chunk, False) + api.qkv4_bytes(chunk)
+        assert need < 2 * 4 * per * head + 2 * api.workspace_bytes(chunk, False) + api.qkv4_bytes(chunk) + 4096
+    assert api.host_staging_bytes(p, 0) == api.host_staging_bytes(p, 5)     # default: ramp up to BH / 8 heads
+    assert api.host_staging_bytes(p, 400) == api.host_staging_bytes(p, 40)  # capped at B*H
+    assert api.host_staging_bytes(p, -1) == 0
+    # B = 2 flattens to B*H heads
+    p2 = api.problem(cfg.replace(B=2, H=4))
+    assert api.host_staging_bytes(p2, 0) == api.host_staging_bytes(api.problem(cfg.replace(H=8)), 1)
+    need = api.host_staging_bytes(p, 0)
+    st = lib.ra_int4_attention_host(ctypes.byref(p), 16, 16, 16, 16, -1, 256, need, None)
+    assert st == api.RA_ERR_INVALID_ARG
+    st = lib.ra_int4_attention_host(ctypes.byref(p), 16, None, 16, 16, 0, 256, need, None)
+    assert st == api.RA_ERR_INVALID_ARG
+    st = lib.ra_int4_attention_host(ctypes.byref(p), 16, 16, 16, 16, 0, 272, need, None)
+    assert st == api.RA_ERR_INVALID_ARG               # staging not 256-byte aligned
+    st = lib.ra_int4_attention_host(ctypes.byref(p), 16, 16, 16, 16, 0, 256, need - 1, None)
+    assert st == api.RA_ERR_WORKSPACE
+    assert b"needs" in lib.ra_last_error_detail()
+    bad = api.problem(cfg.replace(d=64))
+    st = lib.ra_int4_attention_host(ctypes.byref(bad), 16, 16, 16, 16, 0, 256, 1 << 40, None)
+    assert st == api.RA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("name", ["tiny", "half", "wan", "hunyuan"])
 def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
     cfg = synth.CONFIGS[name]
