@@ -52,11 +52,38 @@ __device__ __forceinline__ void h8_to_f(const uint4& u, float (&f)[8]) {
   }
 }
 
-// Symmetric INT4 code: clamp(rne(v / s), -7, 7); 0 when s == 0.
+// Symmetric INT4 code: clamp(rne(v / s), -7, 7) with the IEEE quotient
+// fl(v / s); 0 when s == 0.
 __device__ __forceinline__ int int4_code(float v, float s) {
   if (s == 0.0f) return 0;
   int q = __float2int_rn(__fdiv_rn(v, s));
   return q > 7 ? 7 : (q < -7 ? -7 : q);
+}
+
+// Reciprocal of a block scale for int4_nibble_r: RN(1 / s), or 0 where it
+// would not be a finite normal number (s == 0, or s so small or so large that
+// 1 / s overflows or is subnormal), which sends every element to int4_code.
+__device__ __forceinline__ float code_recip(float s) {
+  const float r = __fdiv_rn(1.0f, s);
+  return (r < 3.0e38f && r > 1.0e-37f) ? r : 0.0f;
+}
+
+// The low nibble of int4_code(v, s) without a division per element, for |v| <= 7 s (1 + 2^-22)
+// (every element of the block whose amax gave s = fl(amax / 7)).  With
+// r = RN(1 / s), |v r - v / s| <= |v| 2^-24 / s <= 7.0 * 2^-24 and
+// |fl(v / s) - v / s| <= 2^-22, so v r is within 6.6e-7 of fl(v / s): the two
+// round to the same integer unless v r lies within that of a half-integer.
+// t = v r + 1.5 * 2^23 rounded once is that integer in the low mantissa bits
+// (exact: |v r| < 7.5); e = v r - rne(v r) tells how close it is to a tie,
+// and elements within 1e-5 of one take the IEEE division.  The result needs
+// no clamp (|v r| < 7.5); its low nibble is the two's-complement code.
+__device__ __forceinline__ uint32_t int4_nibble_r(float v, float s, float r) {
+  constexpr float MAGIC = 12582912.0f;   // 1.5 * 2^23
+  if (r == 0.0f) return (uint32_t)int4_code(v, s) & 0xFu;
+  const float t = __fmaf_rn(v, r, MAGIC);
+  const float e = __fmaf_rn(v, r, -__fsub_rn(t, MAGIC));
+  if (fabsf(e) > 0.49999f) return (uint32_t)int4_code(v, s) & 0xFu;
+  return __float_as_uint(t) & 0xFu;
 }
 
 __device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P, uint32_t site) {
@@ -65,19 +92,42 @@ __device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P,
   return false;
 }
 
+// Where the 4 adjacent pairs of channels c0 .. c0 + 7 find their table
+// entries: entry = base[pp] + pos[axis[pp]] * stride[pp].  Computed once per
+// thread with selects on the segment, so that no per-element lookup indexes
+// the problem's arrays with a run-time segment (which would put them in
+// local memory).
+struct PairTab {
+  int base[4], stride[4], axis[4];
+};
+
+__device__ __forceinline__ int sel3(int s, int a, int b, int c) { return s == 0 ? a : (s == 1 ? b : c); }
+
+__device__ __forceinline__ PairTab pair_tab(const Prob& P, int c0) {
+  PairTab t;
+#pragma unroll
+  for (int pp = 0; pp < 4; ++pp) {
+    const int c = c0 + 2 * pp;
+    const int s = c < P.off[1] ? 0 : (c < P.off[2] ? 1 : 2);
+    const int j = (c - sel3(s, P.off[0], P.off[1], P.off[2])) >> 1;
+    t.base[pp] = sel3(s, P.tab_off[0], P.tab_off[1], P.tab_off[2]) + j;
+    t.stride[pp] = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+    t.axis[pp] = s;
+  }
+  return t;
+}
+
 // RoPE of the 4 adjacent pairs held by one thread (channels c0..c0+7 of
 // token n).  FORM 0: the RoPE rotation (cos, sin); FORM 1: the Interleaved
 // H2 * Rot (alpha, beta); FORM 2: a caller's block times Rot, merged on the
 // host (m00, m01, m10, m11).
 template <int FORM>
-__device__ __forceinline__ void rope8(const Prob& P, const float4* __restrict__ tab, const TokenPos& tp, int c0,
+__device__ __forceinline__ void rope8(const PairTab& pt, const float4* __restrict__ tab, const TokenPos& tp,
                                       const float (&x)[8], float (&y)[8]) {
 #pragma unroll
   for (int pp = 0; pp < 4; ++pp) {
-    const int c = c0 + 2 * pp;
-    const int s = segment_of(P, c);
-    const int j = (c - P.off[s]) >> 1;
-    const float4 t = __ldg(&tab[P.tab_off[s] + tp.p[s] * (P.split[s] >> 1) + j]);
+    const int pos = sel3(pt.axis[pp], tp.p[0], tp.p[1], tp.p[2]);
+    const float4 t = __ldg(&tab[pt.base[pp] + pos * pt.stride[pp]]);
     const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
     if (FORM == 1) {          // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
       y[2 * pp] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
@@ -165,13 +215,14 @@ __global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __ha
   }
   float z[QK_ROWS][8];
   float amax = 0.0f;
+  const PairTab pt = pair_tab(P, c0);
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     float xf[8];
     h8_to_f(raw[i], xf);
     const TokenPos tp = token_pos(P, n < P.N ? n : 0);
-    rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(P, tab, tp, c0, xf, z[i]);
+    rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(pt, tab, tp, xf, z[i]);
   }
   if (HALF_PAIRS) {
 #pragma unroll
@@ -183,11 +234,12 @@ __global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __ha
     for (int e = 0; e < 8; ++e) {
       const int c = c0 + e;
       const int s = segment_of(P, c);
-      const int h = P.split[s] >> 1;
-      const bool first = (c - P.off[s]) < h;
+      const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+      const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
+      const bool first = (c - off) < h;
       float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
       if (ROT == RA_ROT_BLOCKS_HALF)   // block of pair off_s / 2 + i, i = index in the first half
-        r4 = __ldg(&tab[P.n_tab + (P.off[s] >> 1) + (c - P.off[s]) - (first ? 0 : h)]);
+        r4 = __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)]);
 #pragma unroll
       for (int i = 0; i < QK_ROWS; ++i) {
         const int r = r0 + QK_RSTEP * i;
@@ -211,12 +263,13 @@ __global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __ha
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(z[i][e]));
   amax = block_max(amax, red);
   const float s = __fdiv_rn(amax, 7.0f);
+  const float rs = code_recip(s);
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     uint32_t packed = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) packed |= (uint32_t)(int4_code(z[i][e], s) & 0xF) << (4 * e);
+    for (int e = 0; e < 8; ++e) packed |= int4_nibble_r(z[i][e], s, rs) << (4 * e);
     *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = packed;
   }
   if (threadIdx.x == 0) scale[blk] = s;
@@ -273,9 +326,12 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
-  float s[8];
+  float s[8], rs[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
+  for (int e = 0; e < 8; ++e) {
+    s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
+    rs[e] = code_recip(s[e]);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int n = blk * QK_BLOCK + r0 + 8 * i;
@@ -288,7 +344,8 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
     }
     if (P.v_rot) hadamard128(f, g);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) codes[r0 + 8 * i][8 * g + e] = (int8_t)int4_code(f[e], s[e]);
+    for (int e = 0; e < 8; ++e)   // the nibble, sign-extended
+      codes[r0 + 8 * i][8 * g + e] = (int8_t)((int)(int4_nibble_r(f[e], s[e], rs[e]) << 28) >> 28);
   }
   __syncthreads();
   const int c = threadIdx.x;
@@ -340,7 +397,7 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
       if (n < P.N) {
         float xf[8], y[8];
         h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)), xf);
-        rope8<0>(P, tab, token_pos(P, n), c0, xf, y);
+        rope8<0>(pair_tab(P, c0), tab, token_pos(P, n), xf, y);
         __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
