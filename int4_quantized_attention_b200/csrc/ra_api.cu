@@ -105,6 +105,17 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
       P.tab_off[s] = toff;
       toff += npos[s] * (p->split[s] / 2);
     }
+    P.fastdiv = 1;
+    const uint64_t divs[2] = {(uint64_t)(p->W > 0 ? p->W : 1), (uint64_t)(p->W > 0 ? p->W : 1) * (p->Hh > 0 ? p->Hh : 1)};
+    uint32_t mags[2];
+    for (int i = 0; i < 2; ++i) {
+      const uint64_t d = divs[i];
+      const uint64_t m = ((1ull << 32) + d - 1) / d;   // ceil(2^32 / d)
+      mags[i] = m >> 32 ? 0u : (uint32_t)m;            // d = 1: identity
+      if (d > 1 && (uint64_t)nv * (m * d - (1ull << 32)) >= (1ull << 32)) P.fastdiv = 0;
+    }
+    P.m_w = mags[0];
+    P.m_hw = mags[1];
     P.n_tab = toff;
     P.n_tab_all = toff + p->d / 2;
     // what the tables depend on; B and H only size the buffers (checked on the

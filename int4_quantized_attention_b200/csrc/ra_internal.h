@@ -25,6 +25,12 @@ struct Prob {
   int n_tab;                    // RoPE table entries (each: cos, sin, alpha, beta, or for
                                 // BLOCKS_INTERLEAVED the merged m00, m01, m10, m11)
   int n_tab_all;                // n_tab + d/2 pair-block entries (r00, r01, r10, r11)
+  // token -> (f, h, w) without integer division: n / d = umulhi(n, m) for
+  // m = ceil(2^32 / d), exact while n * (m d - 2^32) < 2^32 for every video
+  // token (checked on the host; fastdiv = 0 falls back to / and %); m = 0
+  // stands for d = 1
+  uint32_t m_w, m_hw;           // divisors W and Hh * W
+  int fastdiv;
   int rot;
   int p_mode;                   // ra_p_mode
   int v_rot;                    // 1: Hadamard on V, undone on O (INT4 path)
