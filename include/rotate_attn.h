@@ -194,15 +194,19 @@ size_t ra_host_staging_bytes(const ra_problem *p, int heads_per_chunk);
  * chunks of consecutive heads, each chunk as a problem of its own with B = 1
  * (every step of the path is independent per head, so the results are
  * bit-identical to the device-buffer calls).  heads_per_chunk > 0: chunks of
- * that many heads; 0: chunks of 1, 2, 3, ... heads growing to about B*H/8,
- * so that the kernels start after a one-head copy.  While chunk c is computed on `stream`, the inputs
- * of chunk c+1 are copied in and the output of chunk c-1 is copied out on
- * two streams the call creates and destroys.  The copies overlap only if the
- * host buffers are page-locked (cudaHostAlloc / cudaHostRegister); pageable
- * buffers give the same result without the overlap.
+ * that many heads; 0: chunks of about B*H/8 heads, entered and left by ramps
+ * of 1, 2, 3, ... heads, so that the kernels start after a one-head copy and
+ * the last copy back is of one head.  While chunk c is computed, the inputs
+ * of chunk c+1 are copied in and the output of chunk c-1 is copied out;
+ * chunks alternate between `stream` and a second compute stream so that the
+ * kernels of chunk c+1 start on the SMs chunk c's last wave leaves idle.  The
+ * call creates and destroys its three extra streams and six events.  The
+ * copies overlap only if the host buffers are page-locked (cudaHostAlloc /
+ * cudaHostRegister); pageable buffers give the same result without the
+ * overlap.
  * staging: device memory owned by the caller, 256-byte aligned, at least
- * ra_host_staging_bytes(p, heads_per_chunk) bytes: two slots of q, k, v, o
- * for the largest chunk plus the quantised tensors and workspace of one.  The
+ * ra_host_staging_bytes(p, heads_per_chunk) bytes: two slots, each with q, k,
+ * v, o, the quantised tensors and a workspace for the largest chunk.  The
  * call blocks until o is written and the device error words are checked,
  * so it returns any status ra_check_device_error can.  The staging buffer
  * must not be used by other work while the call runs. */

@@ -4,15 +4,18 @@
 // Heads are independent in every step of the path (Q/K blocks, V channel
 // scales and the attention all live inside one (b, h)), so the flattened
 // B*H heads are cut into chunks of consecutive heads, each a problem of its
-// own with B = 1.  Three streams form a pipeline over the chunks:
+// own with B = 1.  Four streams form a pipeline over the chunks:
 //
-//   copy-in stream : q, k, v of chunk c, host -> slot c % 2
-//   caller's stream: prologue + INT4 attention of chunk c (slot c % 2)
-//   copy-out stream: o of chunk c, slot c % 2 -> host
+//   copy-in stream   : q, k, v of chunk c, host -> slot c % 2
+//   compute lane c%2 : prologue + INT4 attention of chunk c (slot c % 2);
+//                      lane 0 is the caller's stream, lane 1 one of ours
+//   copy-out stream  : o of chunk c, slot c % 2 -> host
 //
 // so that the host->device copy of chunk c+1 and the device->host copy of
-// chunk c-1 run on the copy engines while chunk c is computed.  Events order
-// the reuse of the two slots.  The call blocks until o is written.
+// chunk c-1 run on the copy engines while chunk c is computed, and the
+// kernels of chunk c+1 fill the SMs that the last wave of chunk c leaves idle
+// (each slot has its own quantised tensors and workspace).  Events order the
+// reuse of the two slots.  The call blocks until o is written.
 #include <algorithm>
 #include <cstdio>
 #include <vector>
@@ -30,15 +33,16 @@ struct HostPlan {
   int BH, per;                // flattened heads; the largest chunk
   ra_problem chunk;           // B = 1, H = per (sizes the regions below)
   size_t head_bytes;          // one head of one fp16 tensor: N * 128 * 2
-  size_t ws, qkv4, slot;      // region sizes (256-aligned)
-  size_t off_qkv4, off_slots, total;
+  size_t ws, qkv4, io;        // per-slot region sizes (256-aligned)
+  size_t slot, total;         // one slot: workspace, quantised tensors, q, k, v, o
 };
 
 // Chunk sizes.  Given heads_per_chunk > 0: equal chunks (the last one takes
-// the remainder).  Given 0: chunks of about B*H/8 heads, reached by a ramp
-// 1, 2, 3, ... so that the first kernels wait only for a one-head copy (the
-// copy of a head takes about 3/4 of its compute, so each chunk's copy-in
-// hides behind the previous chunk's kernels when sizes grow by at most 4/3).
+// the remainder).  Given 0: chunks of about B*H/8 heads, entered and left by
+// ramps 1, 2, 3, ... so that the first kernels wait only for a one-head copy
+// and the last copy-out is of one head (a head's copy-in takes about 3/4 of
+// its compute, so each chunk's copy-in hides behind the previous chunk's
+// kernels when sizes grow by at most 4/3).
 void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
   out.clear();
   if (heads_per_chunk > 0) {
@@ -46,13 +50,25 @@ void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
     return;
   }
   const int per = (BH + kDefaultChunks - 1) / kDefaultChunks;
-  int done = 0, next = 1;
-  while (done < BH) {
-    const int c = std::min(std::min(next, per), BH - done);
-    out.push_back(c);
-    done += c;
-    next = std::max(next + 1, (4 * c) / 3);
+  std::vector<int> ramp;
+  int ramp_sum = 0;
+  for (int next = 1; next < per; next = std::max(next + 1, (4 * next) / 3)) {
+    ramp.push_back(next);
+    ramp_sum += next;
   }
+  if (2 * ramp_sum > BH) {   // too few heads for both ramps: ramp up only
+    int done = 0, next = 1;
+    while (done < BH) {
+      const int c = std::min(std::min(next, per), BH - done);
+      out.push_back(c);
+      done += c;
+      next = std::max(next + 1, (4 * c) / 3);
+    }
+    return;
+  }
+  out = ramp;
+  for (int mid = BH - 2 * ramp_sum; mid > 0; mid -= per) out.push_back(std::min(per, mid));
+  out.insert(out.end(), ramp.rbegin(), ramp.rend());
 }
 
 ra_status plan(const ra_problem* p, int heads_per_chunk, HostPlan* hp) {
@@ -73,10 +89,9 @@ ra_status plan(const ra_problem* p, int heads_per_chunk, HostPlan* hp) {
   h.head_bytes = (size_t)P.N * ra::D * 2;
   h.ws = ra::align256(ra_workspace_bytes(&h.chunk, 0));
   h.qkv4 = ra::align256(ra_qkv4_bytes(&h.chunk));
-  h.slot = ra::align256(4 * h.per * h.head_bytes);    // q, k, v, o of one chunk
-  h.off_qkv4 = h.ws;
-  h.off_slots = h.off_qkv4 + h.qkv4;
-  h.total = h.off_slots + 2 * h.slot;
+  h.io = ra::align256(4 * h.per * h.head_bytes);    // q, k, v, o of one chunk
+  h.slot = h.ws + h.qkv4 + h.io;
+  h.total = 2 * h.slot;
   return RA_OK;
 }
 
@@ -90,7 +105,7 @@ ra_status cuda_err(cudaError_t e, const char* what) {
 
 // Streams and events of one call, released on every path out of it.
 struct Pipeline {
-  cudaStream_t in = nullptr, out = nullptr;
+  cudaStream_t in = nullptr, out = nullptr, lane1 = nullptr;
   cudaEvent_t loaded[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr}, stored[2] = {nullptr, nullptr};
   ~Pipeline() {
     for (int i = 0; i < 2; ++i) {
@@ -100,10 +115,12 @@ struct Pipeline {
     }
     if (in) cudaStreamDestroy(in);
     if (out) cudaStreamDestroy(out);
+    if (lane1) cudaStreamDestroy(lane1);
   }
   cudaError_t create() {
     cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&lane1, cudaStreamNonBlocking);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&loaded[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[i], cudaEventDisableTiming);
@@ -143,15 +160,17 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(staging);
-  void* ws = base;
+  void* ws[2] = {base, base + h.slot};
 
-  // Tables and signature (synchronises `stream`); the signature does not
-  // cover B or H, so this workspace serves every chunk.
-  if ((st = ra_prepare(&h.chunk, ws, h.ws, stream)) != RA_OK) return st;
+  // Tables and signature of both slots' workspaces (synchronises `stream`);
+  // the signature does not cover B or H, so each serves every chunk size.
+  for (int i = 0; i < 2; ++i)
+    if ((st = ra_prepare(&h.chunk, ws[i], h.ws, stream)) != RA_OK) return st;
 
   Pipeline pl;
   cudaError_t e = pl.create();
   if (e != cudaSuccess) return cuda_err(e, "stream/event creation");
+  cudaStream_t lane[2] = {s, pl.lane1};
 
   const char* qh = static_cast<const char*>(q);
   const char* kh = static_cast<const char*>(k);
@@ -162,25 +181,27 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
     const int sl = (int)(c & 1);
     ra_problem cp = h.chunk;
     cp.H = h.heads[c];
+    char* slot = base + sl * h.slot;
     ra_qkv4 qkv;
-    if ((st = ra_qkv4_bind(&cp, base + h.off_qkv4, h.qkv4, &qkv)) != RA_OK) break;
+    if ((st = ra_qkv4_bind(&cp, slot + h.ws, h.qkv4, &qkv)) != RA_OK) break;
     const size_t n = (size_t)cp.H * h.head_bytes;
-    char* slot = base + h.off_slots + sl * h.slot;
-    char *qd = slot, *kd = slot + n, *vd = slot + 2 * n, *od = slot + 3 * n;
+    char* io = slot + h.ws + h.qkv4;
+    char *qd = io, *kd = io + n, *vd = io + 2 * n, *od = io + 3 * n;
 
-    // copy-in: the slot's inputs are free once chunk c-2 has been computed
+    // copy-in: the slot is free once chunk c-2 has been computed
     if (c >= 2 && (e = cudaStreamWaitEvent(pl.in, pl.computed[sl], 0)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(qd, qh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(kd, kh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(vd, vh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaEventRecord(pl.loaded[sl], pl.in)) != cudaSuccess) break;
 
-    // compute: inputs loaded, and the slot's output read back (chunk c-2)
-    if ((e = cudaStreamWaitEvent(s, pl.loaded[sl], 0)) != cudaSuccess) break;
-    if (c >= 2 && (e = cudaStreamWaitEvent(s, pl.stored[sl], 0)) != cudaSuccess) break;
-    if ((st = ra_rotate_quantize_qkv(&cp, qd, kd, vd, &qkv, ws, h.ws, stream)) != RA_OK) break;
-    if ((st = ra_int4_attention_fwd(&cp, &qkv, od, ws, h.ws, stream)) != RA_OK) break;
-    if ((e = cudaEventRecord(pl.computed[sl], s)) != cudaSuccess) break;
+    // compute on lane c % 2 (after chunk c-2 on the same lane): inputs
+    // loaded, and the slot's output read back (chunk c-2)
+    if ((e = cudaStreamWaitEvent(lane[sl], pl.loaded[sl], 0)) != cudaSuccess) break;
+    if (c >= 2 && (e = cudaStreamWaitEvent(lane[sl], pl.stored[sl], 0)) != cudaSuccess) break;
+    if ((st = ra_rotate_quantize_qkv(&cp, qd, kd, vd, &qkv, ws[sl], h.ws, lane[sl])) != RA_OK) break;
+    if ((st = ra_int4_attention_fwd(&cp, &qkv, od, ws[sl], h.ws, lane[sl])) != RA_OK) break;
+    if ((e = cudaEventRecord(pl.computed[sl], lane[sl])) != cudaSuccess) break;
 
     // copy-out
     if ((e = cudaStreamWaitEvent(pl.out, pl.computed[sl], 0)) != cudaSuccess) break;
@@ -188,10 +209,12 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
     if ((e = cudaEventRecord(pl.stored[sl], pl.out)) != cudaSuccess) break;
     off += n;
   }
-  // Join both copy streams into the caller's stream, then wait for all of it,
+  // Join the other streams into the caller's stream, then wait for all of it,
   // also on an error path (nothing may still use the staging buffer on return).
   cudaError_t j = cudaEventRecord(pl.loaded[0], pl.in);
   if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.loaded[0], 0);
+  if (j == cudaSuccess) j = cudaEventRecord(pl.computed[1], pl.lane1);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.computed[1], 0);
   if (j == cudaSuccess) j = cudaEventRecord(pl.stored[0], pl.out);
   if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.stored[0], 0);
   cudaError_t w = cudaStreamSynchronize(s);
@@ -199,7 +222,8 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   if (e != cudaSuccess) return cuda_err(e, "pipeline enqueue");
   if (j != cudaSuccess) return cuda_err(j, "pipeline join");
   if (w != cudaSuccess) return cuda_err(w, "pipeline synchronize");
-  return ra_check_device_error(ws, stream);
+  if ((st = ra_check_device_error(ws[0], stream)) != RA_OK) return st;
+  return ra_check_device_error(ws[1], stream);
 }
 
 }  // extern "C"

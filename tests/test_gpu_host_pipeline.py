@@ -39,6 +39,9 @@ CASES = [
     ("tiny", {"B": 2, "H": 3}, (0, 4, 6)),
     ("tiny", {"B": 2, "H": 20}, (0, 7)),    # default ramp 1, 2, 3, 4, 5, 5, ... over 40 heads
     ("wan", {"H": 5}, (2,)),                  # full Wan sequence, ragged last tile, tail of 1 head
+    # the options ride along: caller pair blocks (Half), V Hadamard, symmetric P map
+    ("half", {"rot": "blocks_half", "blocks": synth.random_pair_blocks(3), "v_rot": 1, "p_mode": "symmetric"},
+     (0, 3)),
 ]
 
 
