@@ -322,21 +322,16 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
 
 // One CTA = one 64-token block of V of one head: codes with the per-channel
 // scale, transposed packing (channel-major, two tokens per byte) and the
-// block's column sums.  Thread (g, t) = (tid % 16, tid / 16) holds channels
-// 8g .. 8g + 7 of the consecutive tokens 8t .. 8t + 7, so it packs the eight
-// nibbles of each of its channels into that channel's word t in registers;
-// shared memory only regroups the words and partial sums by channel for
-// coalesced stores.
+// block's column sums.
 __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
                                                       const uint32_t* __restrict__ vamax,
                                                       uint8_t* __restrict__ v4t, float* __restrict__ sv,
                                                       int32_t* __restrict__ vsum,
                                                       const WsHeader* __restrict__ hdr) {
-  __shared__ uint32_t words[D][9];   // [channel][token group t], padded
-  __shared__ int sums[8][D];         // [token group][channel]
+  __shared__ int8_t codes[QK_BLOCK][D + 16];
   if (!signature_ok(hdr, P, 0x300)) return;
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const int g = threadIdx.x & 15, t = threadIdx.x >> 4;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
   float s[8], rs[8];
 #pragma unroll
@@ -344,11 +339,9 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
     s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
     rs[e] = code_recip(s[e]);
   }
-  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  int sum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const int n = blk * QK_BLOCK + 8 * t + k;
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
     float f[8];
     if (n < P.N) {
       h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
@@ -356,30 +349,32 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = 0.0f;
     }
-    if (P.v_rot) hadamard128(f, g);   // the 16 lanes of a token are one half-warp
+    if (P.v_rot) hadamard128(f, g);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t nib = int4_nibble_r(f[e], s[e], rs[e]);
-      w[e] |= nib << (4 * k);
-      sum[e] += (int)(nib << 28) >> 28;
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    words[8 * g + e][t] = w[e];
-    sums[t][8 * g + e] = sum[e];
+    for (int e = 0; e < 8; ++e)   // the nibble, sign-extended
+      codes[r0 + 8 * i][8 * g + e] = (int8_t)((int)(int4_nibble_r(f[e], s[e], rs[e]) << 28) >> 28);
   }
   __syncthreads();
   const int c = threadIdx.x;
-  int total = 0;
+  uint32_t w[8];
+  int sum = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) total += sums[i][c];
+  for (int t = 0; t < 8; ++t) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int code = codes[8 * t + e][c];
+      sum += code;
+      word |= (uint32_t)(code & 0xF) << (4 * e);
+    }
+    w[t] = word;
+  }
   // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
   uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
                                         (size_t)(blk % 2) * (QK_BLOCK / 2));
-  dst[0] = make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
-  dst[1] = make_uint4(words[c][4], words[c][5], words[c][6], words[c][7]);
-  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = total;
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
   if (blk == 0) sv[(size_t)bh * D + c] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
 }
 
