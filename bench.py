@@ -314,7 +314,8 @@ def our_arm(args, cfg, rank, world):
         "e2e": {"value": aggregate_tops(world, ops, ms_e2e), "unit": "TOPS", "ms_per_step": ms_e2e,
                 "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2,
                 "api": "ra_int4_attention_host (pinned host q, k, v, o; copies overlapped over head chunks)",
-                "heads_per_chunk": args.chunk_heads or -(-BH // 8),
+                "chunks": (f"{args.chunk_heads} heads each" if args.chunk_heads else
+                           f"library default: ramp 1, 2, 3, ... up to {-(-BH // 8)} heads and back down"),
                 "serial_ms_per_step": ms_e2e_serial},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
