@@ -343,12 +343,4 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
-// K-major operand without swizzle: 8-row x 16-byte core matrices, rows 16
-// bytes apart; 8-row groups 128 bytes apart (stride byte offset), the two
-// 8-element K halves 2048 bytes apart (leading byte offset); K = 16 bf16.
-__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(2048u >> 4) << 16) | ((uint64_t)(128u >> 4) << 32) |
-         ((uint64_t)1u << 46);
-}
-
 }  // namespace ra
