@@ -268,6 +268,11 @@ ra_status ra_debug_int4_tile(const ra_problem *p, const ra_qkv4 *in, int bh, int
                              int32_t *s_out, int8_t *p_out, void *workspace, size_t workspace_bytes,
                              ra_stream stream);
 
+/* The chunk sizes (heads per chunk, in order) ra_int4_attention_host would
+ * use: writes min(count, max_chunks) of them to sizes (may be NULL) and
+ * returns the count, or -1 for an invalid problem or heads_per_chunk < 0. */
+int ra_host_chunks(const ra_problem *p, int heads_per_chunk, int *sizes, int max_chunks);
+
 /* Sets the wall-clock limit of every bounded device-side wait, in
  * microseconds (0 restores the default of 2 s); a test sets 1 and runs
  * ra_debug_timeout_probe, whose kernel waits on a barrier that nothing arms

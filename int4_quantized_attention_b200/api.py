@@ -61,6 +61,7 @@ _SIGNATURES = {
     "ra_check_device_error": (ctypes.c_int, [_V, _V]),
     "ra_host_staging_bytes": (_SZ, [_P, ctypes.c_int]),
     "ra_int4_attention_host": (ctypes.c_int, [_P, _V, _V, _V, _V, ctypes.c_int, _V, _SZ, _V]),
+    "ra_host_chunks": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
     "ra_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ra_last_error_detail": (ctypes.c_char_p, []),
     "ra_tables_floats": (_SZ, [_P]),
@@ -179,6 +180,16 @@ def fp16_attention_fwd(p: Problem, q, k, v, o, workspace, stream=None) -> None:
 
 def host_staging_bytes(p: Problem, heads_per_chunk: int = 0) -> int:
     return lib().ra_host_staging_bytes(ctypes.byref(p), heads_per_chunk)
+
+
+def host_chunks(p: Problem, heads_per_chunk: int = 0) -> list:
+    """Heads per chunk, in order, of ra_int4_attention_host's pipeline."""
+    n = lib().ra_host_chunks(ctypes.byref(p), heads_per_chunk, None, 0)
+    if n < 0:
+        _check("ra_host_chunks", RA_ERR_INVALID_ARG)
+    out = (ctypes.c_int * max(n, 1))()
+    lib().ra_host_chunks(ctypes.byref(p), heads_per_chunk, out, n)
+    return list(out[:n])
 
 
 def int4_attention_host(p: Problem, q, k, v, o, staging, heads_per_chunk: int = 0, stream=None) -> None:

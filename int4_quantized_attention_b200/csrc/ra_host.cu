@@ -66,8 +66,16 @@ void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
     }
     return;
   }
+  // the middle (chunks of at most per heads, balanced) must not dip below the
+  // ramp's top: hand the top steps of both ramps to the middle until it fits
+  int mid = BH - 2 * ramp_sum;
+  while (!ramp.empty() && mid < ramp.back()) {
+    mid += 2 * ramp.back();
+    ramp.pop_back();
+  }
   out = ramp;
-  for (int mid = BH - 2 * ramp_sum; mid > 0; mid -= per) out.push_back(std::min(per, mid));
+  const int n_mid = (mid + per - 1) / per;
+  for (int i = 0; i < n_mid; ++i) out.push_back(mid / n_mid + (i < mid % n_mid ? 1 : 0));
   out.insert(out.end(), ramp.rbegin(), ramp.rend());
 }
 
@@ -137,6 +145,15 @@ extern "C" {
 size_t ra_host_staging_bytes(const ra_problem* p, int heads_per_chunk) {
   HostPlan h;
   return plan(p, heads_per_chunk, &h) == RA_OK ? h.total : 0;
+}
+
+int ra_host_chunks(const ra_problem* p, int heads_per_chunk, int* sizes, int max_chunks) {
+  HostPlan h;
+  if (plan(p, heads_per_chunk, &h) != RA_OK) return -1;
+  const int n = (int)h.heads.size();
+  if (sizes != nullptr)
+    for (int i = 0; i < n && i < max_chunks; ++i) sizes[i] = h.heads[i];
+  return n;
 }
 
 ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void* k, const void* v, void* o,

@@ -164,6 +164,32 @@ def test_host_entry_plan_and_argument_checks(lib):
     assert st == api.RA_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("BH", [1, 2, 3, 5, 8, 9, 16, 24, 40, 41, 64, 100, 333])
+def test_host_chunk_schedule(lib, BH):
+    """The default schedule covers the B*H heads in order, never exceeds
+    ceil(B*H/8) heads a chunk, starts and (when there is room for both ramps)
+    ends with one head, and grows or shrinks by at most 4/3 (+1) per step;
+    an explicit size gives equal chunks and a remainder."""
+    p = api.problem(synth.CONFIGS["tiny"].replace(B=1, H=BH))
+    per = -(-BH // 8)
+    c = api.host_chunks(p, 0)
+    assert sum(c) == BH and min(c) >= 1 and max(c) <= per and c[0] == 1
+    for a, b in zip(c, c[1:]):   # growth the copy-in can hide behind the previous chunk's kernels
+        assert b <= max(a + 1, 4 * a // 3)
+    if BH >= 8:
+        assert c[-1] == 1        # room for the down ramp: the last copy back is of one head
+    assert api.host_chunks(p, 7) == [7] * (BH // 7) + ([BH % 7] if BH % 7 else [])
+    assert api.host_chunks(p, 10 ** 6) == [BH]
+    assert lib.ra_host_chunks(ctypes.byref(p), -1, None, 0) == -1
+    # the staging size follows the largest chunk
+    assert api.host_staging_bytes(p, 0) == api.host_staging_bytes(p, max(c))
+
+
+def test_host_chunk_schedule_wan_and_hunyuan(lib):
+    assert api.host_chunks(api.problem(synth.CONFIGS["wan"])) == [1, 2, 3, 4, 5, 5, 5, 5, 4, 3, 2, 1]
+    assert api.host_chunks(api.problem(synth.CONFIGS["hunyuan"])) == [1, 2, 3, 3, 3, 3, 3, 3, 2, 1]
+
+
 @pytest.mark.parametrize("name", ["tiny", "half", "wan", "hunyuan"])
 def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
     cfg = synth.CONFIGS[name]
