@@ -58,6 +58,8 @@ def lib():
         _lib.orc_p_code.argtypes = [ctypes.c_float]
         _lib.orc_p_code_sym.restype = ctypes.c_int
         _lib.orc_p_code_sym.argtypes = [ctypes.c_float]
+        _lib.orc_p_weight.restype = ctypes.c_int
+        _lib.orc_p_weight.argtypes = [ctypes.c_float, ctypes.c_int]
         _lib.orc_rope_angle.restype = ctypes.c_double
         _lib.orc_seq_len.restype = ctypes.c_int
         _lib.orc_seq_pad.restype = ctypes.c_int
@@ -114,6 +116,11 @@ def p_code(P: float) -> int:
 
 def p_code_sym(P: float) -> int:
     return lib().orc_p_code_sym(ctypes.c_float(P))
+
+
+def p_weight(x: float, levels: int = 15) -> int:
+    """rne(levels * 2^x) for the fp32 exponent x (the quantised path's P weight)."""
+    return lib().orc_p_weight(ctypes.c_float(x), levels)
 
 
 def _quant_mode(cfg, quant_p) -> int:

@@ -25,9 +25,11 @@
  *
  * Precision: every step that decides an integer (a Q/K/V code, a P code)
  * is taken in IEEE fp32 with no FMA contraction (build with
- * -ffp-contract=off), because that is the precision the CUDA path decides in;
- * integer products are exact (int32/int64); the running accumulators of the
- * online softmax are float64.
+ * -ffp-contract=off; the one fused multiply-add, in the P exponent, is an
+ * explicit fmaf), because that is the precision the CUDA path decides in;
+ * the P code itself is then exact for its fp32 exponent; integer products are
+ * exact (int32/int64); the running accumulators of the online softmax are
+ * float64.
  */
 #include <math.h>
 #include <stdint.h>
@@ -341,17 +343,29 @@ int orc_p_code(float P) { return (int)nearbyintf(15.0f * P) - 8; }
  * no zero-point. */
 int orc_p_code_sym(float P) { return (int)nearbyintf(7.0f * P); }
 
+/* The P weight w = code + zero-point of the quantised path, taken from the
+ * exponent in log2 units: w = rne(levels * 2^x) with P = 2^x, levels = 15
+ * for the range-optimised map (code = w - 8) and 7 for the symmetric one
+ * (code = w).  READING: the pages fix no precision for P = exp(s - m); the
+ * code is decided for the fp32 exponent x, exactly: levels * 2^x is
+ * evaluated in float64 (exact to ~1e-16 relative, far below the distance of
+ * any 2^x with fp32 x from a half-integer, except x = -1 where
+ * 15 * 2^-1 = 7.5 exactly and the round-half-to-even rint gives 8). */
+int orc_p_weight(float x, int levels) { return (int)rint((double)levels * exp2((double)x)); }
+
 /* One query row i of the INT4 attention (one head), T_kv = `tile` keys per
  * step of the online softmax (128 for the method as built).
  *
  * Per tile j (keys [n0, n1)):
  *   S[n]  = sum_c q_code[i,c] k_code[n,c]                         (int32)
- *   s[n]  = S[n] * (s_Q[i/64] * s_K[n/64]) * (1/sqrt d)            (fp32)
- *   m_j   = max(m_{j-1}, max_n s[n])                               (fp32)
- *   P[n]  = exp(s[n] - m_j);  code[n] = rne(15 P) - 8              (fp32)
+ *   s[n]  = S[n] * s_Q[i/64] * s_K[n/64] / sqrt d, taken in log2 units:
+ *           t[n] = S[n] * c_b with c_b = (s_Q[i/64] log2(e) / sqrt d) s_K[b] (fp32)
+ *   m_j   = max(m_{j-1}, max_n t[n])                               (fp32)
+ *   P[n]  = exp(s[n] - s_max) = 2^x[n], x[n] = S[n] c_b - m_j      (fp32, one rounding)
+ *   code[n] = rne(15 P) - 8, decided exactly for that x            (float64)
  *   PV[c] = sum_n code[n] v_code[n,c] + 8 colsum_j[c]              (int64)
  *   L     = sum_n (code[n] + 8)                                    (int64)
- *   acc   = acc * exp(m_{j-1} - m_j) + PV;  l = l * exp(..) + L    (float64)
+ *   acc   = acc * 2^(m_{j-1} - m_j) + PV;  l = l * 2^(..) + L     (float64)
  * O[i,c] = acc[c] * s_V[c] / l, rounded to fp16; the common 1/15 cancels.
  * READINGS: the standard 1/sqrt(d) softmax scale applies to the dequantised
  * logits; the normaliser uses the dequantised codes (keeps O a convex
@@ -359,8 +373,9 @@ int orc_p_code_sym(float P) { return (int)nearbyintf(7.0f * P); }
  *
  * quant_p = 1: the range-optimised code above.  quant_p = 2: the symmetric
  * code rne(7 P) instead, with no zero-point term and L = sum code.
- * quant_p = 0 replaces the P code by the exact P (float64) and drops the
- * zero-point, for checking the loop against two-pass softmax attention.
+ * quant_p = 0 replaces the P code by the exact P (float64, natural-log
+ * units, s = fl(fl(S fl(s_Q s_K)) / sqrt d)) and drops the zero-point, for
+ * checking the loop against two-pass softmax attention.
  * Optional outputs: o64 [d] (float64 before the fp16 rounding); for tile
  * index dbg_tile >= 0, dbg_S [tile] and dbg_P [tile] (S and P codes of that
  * tile, -128 where the key is past N).
@@ -372,6 +387,15 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
 {
     int N = orc_seq_len(p), d = p->d;
     const float inv_sqrt_d = (float)(1.0 / sqrt((double)d));
+    /* quantised P: log2 units in fp32, the precision the CUDA path decides
+     * in: K = fl(fl(log2 e) / fl(sqrt d)), per 64-key block b the factor
+     * c_b = fl(fl(s_Q[i/64] K) s_K[b]), the dequantised logit t = fl(S c_b)
+     * (s log2 e), the running max m of t, the exponent x = fl(S c_b - m)
+     * rounded once (a fused multiply-add), and w = rne(levels 2^x) exactly
+     * (orc_p_weight).  With P = 2^x this is P = exp(s - m). */
+    const float log2e_f = (float)M_LOG2E, sqrt_d_f = (float)sqrt((double)d);
+    const float K_log2 = log2e_f / sqrt_d_f;
+    const float kq = qs[i / QK_BLOCK] * K_log2;
     float m = -INFINITY;
     double *acc = (double *)calloc((size_t)d, sizeof(double));
     double l = 0.0;
@@ -386,9 +410,14 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
             int32_t acc_s = 0;
             for (int c = 0; c < d; ++c) acc_s += (int32_t)qrow[c] * (int32_t)kc[(size_t)n * d + c];
             S[n - n0] = acc_s;
-            float sc = qs[i / QK_BLOCK] * ks[n / QK_BLOCK];
-            float t = (float)acc_s * sc;
-            float s = t * inv_sqrt_d;
+            float s;
+            if (quant_p) {
+                s = (float)acc_s * (kq * ks[n / QK_BLOCK]);   /* log2 units */
+            } else {
+                float sc = qs[i / QK_BLOCK] * ks[n / QK_BLOCK];
+                float t = (float)acc_s * sc;
+                s = t * inv_sqrt_d;
+            }
             sl[n - n0] = s;
             if (s > tmax) tmax = s;
         }
@@ -400,8 +429,8 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
             int64_t Li = 0;
             const int zp = quant_p == 2 ? 0 : 8;
             for (int n = n0; n < n1; ++n) {
-                float P = expf(sl[n - n0] - m_new);
-                int code = quant_p == 2 ? orc_p_code_sym(P) : orc_p_code(P);
+                float x = fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m_new);
+                int code = quant_p == 2 ? orc_p_weight(x, 7) : orc_p_weight(x, 15) - 8;
                 Li += code + zp;
                 for (int c = 0; c < d; ++c) pvi[c] += (int64_t)code * vc[(size_t)n * d + c];
                 if (j == dbg_tile && dbg_P) dbg_P[n - n0] = (int8_t)code;
@@ -425,7 +454,7 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
                 if (dbg_P && n0 + n >= n1) dbg_P[n] = -128;
             }
         }
-        double alpha = (j == 0) ? 0.0 : exp((double)m - (double)m_new);
+        double alpha = (j == 0) ? 0.0 : quant_p ? exp2((double)m - (double)m_new) : exp((double)m - (double)m_new);
         for (int c = 0; c < d; ++c) acc[c] = acc[c] * alpha + pv[c];
         l = l * alpha + L;
         m = m_new;

@@ -32,6 +32,17 @@ MUTANTS = {
     "hadamard_skips_stride_1": ("for (int h = 1; h < d; h <<= 1)", "for (int h = 2; h < d; h <<= 1)"),
     "p_sym_scale_8": ("nearbyintf(7.0f * P)", "nearbyintf(8.0f * P)"),
     "sym_keeps_zero_point": ("const int zp = quant_p == 2 ? 0 : 8;", "const int zp = 8;"),
+    # the quantised path's exponent in log2 units
+    "log2_scale_index": ("(float)acc_s * (kq * ks[n / QK_BLOCK])", "(float)acc_s * (kq * ks[i / QK_BLOCK])"),
+    "exponent_scale_index": ("fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m_new)",
+                             "fmaf((float)S[n - n0], kq * ks[n0 / QK_BLOCK], -m_new)"),
+    "natural_not_log2": ("const float log2e_f = (float)M_LOG2E", "const float log2e_f = 1.0f"),
+    "log2_softmax_scale": ("const float K_log2 = log2e_f / sqrt_d_f;", "const float K_log2 = log2e_f / (float)d;"),
+    "exponent_drops_max": ("fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m_new)",
+                           "fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m)"),
+    "rescale_sign_log2": ("exp2((double)m - (double)m_new)", "exp2((double)m_new - (double)m)"),
+    "p_weight_levels_16": ("orc_p_weight(x, 15) - 8", "orc_p_weight(x, 16) - 8"),
+    "p_weight_floor": ("(int)rint((double)levels * exp2((double)x))", "(int)floor((double)levels * exp2((double)x))"),
 }
 
 

@@ -62,6 +62,45 @@ def test_p_map_symmetric_golden(oracle_mod):
     assert oracle_mod.p_code_sym(0.5 / 7) == 0 and oracle_mod.p_code_sym(1.5 / 7) == 2
 
 
+def test_p_weight_matches_the_p_map(oracle_mod):
+    """The quantised path decides w = rne(levels 2^x) from the exponent in log2
+    units (P = 2^x): it must agree with the golden P maps, code = w - 8
+    (range-optimised, 15 levels) or w (symmetric, 7 levels), at the endpoints,
+    at every exact level, and wherever levels * P is not within float
+    rounding of a half-integer; it is monotone, and the one exact tie,
+    x = -1 (15 / 2 = 7.5), rounds half to even."""
+    g = json.load(open(os.path.join(GOLDEN, "p_map.json")))
+    gs = json.load(open(os.path.join(GOLDEN, "p_map_symmetric.json")))
+    for golden, levels, zp in ((g, 15, 8), (gs, 7, 0)):
+        for P, code in golden["endpoints"]:
+            x = -math.inf if P == 0.0 else math.log2(P)
+            assert oracle_mod.p_weight(x, levels) - zp == code
+        for kk in range(1, levels + 1):
+            assert oracle_mod.p_weight(float(np.float32(math.log2(kk / levels))), levels) == kk
+    assert oracle_mod.p_weight(-1.0, 15) == 8 and oracle_mod.p_weight(-1.0, 7) == 4   # 7.5 -> 8, 3.5 -> 4
+    xs = np.linspace(-8.0, 0.0, 40001, dtype=np.float32)
+    w = np.array([oracle_mod.p_weight(float(x), 15) for x in xs])
+    assert np.all(np.diff(w) >= 0) and w[0] == 0 and w[-1] == 15
+    exact = 15.0 * np.exp2(xs.astype(np.float64))
+    away = np.abs(exact - np.floor(exact) - 0.5) > 1e-5
+    codes = np.array([oracle_mod.p_code(float(np.exp2(np.float64(x)))) for x in xs])
+    assert np.array_equal(w[away], codes[away] + 8)
+    assert np.max(np.abs(w / 15.0 - np.exp2(xs.astype(np.float64)))) <= 1.0 / 30 + 1e-12
+    # at every rounding boundary, float by float: w steps up exactly at the
+    # first fp32 x with levels * 2^x >= k + 1/2 (extended precision here)
+    ld = np.longdouble
+    for levels in (15, 7):
+        for k in range(levels):
+            edge = np.log2(ld(2 * k + 1) / ld(2 * levels))
+            x = np.float32(edge)
+            for _ in range(3):
+                x = np.nextafter(x, np.float32(-np.inf))
+            for _ in range(7):
+                want = k + 1 if ld(x) >= edge else k
+                assert oracle_mod.p_weight(float(x), levels) == want, (levels, k, float(x))
+                x = np.nextafter(x, np.float32(np.inf))
+
+
 def test_schedule_golden():
     g = json.load(open(os.path.join(GOLDEN, "schedule.json")))
     for c in g["cases"]:
