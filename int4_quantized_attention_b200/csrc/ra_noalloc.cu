@@ -31,6 +31,20 @@ std::mutex g_mutex;
 void* g_scratch_dev[kMaxDevices] = {};                        // device address, per device
 alignas(16) unsigned char g_stage[RA_NOALLOC_SCRATCH_BYTES];  // host staging of header + tables
 
+// The array's device address on device `dev` (current), looked up on the
+// device's first call and kept; a failed call drops it, so it is looked up
+// again after a device reset.  Caller holds g_mutex.
+cudaError_t scratch_address(int dev, char** out) {
+  if (g_scratch_dev[dev] == nullptr) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_dev[dev] = ptr;
+  }
+  *out = static_cast<char*>(g_scratch_dev[dev]);
+  return cudaSuccess;
+}
+
 ra_status cuda_err(cudaError_t e, const char* what) {
   char msg[200];
   snprintf(msg, sizeof(msg), "%s: %s", what, cudaGetErrorString(e));
@@ -78,15 +92,8 @@ extern "C" ra_status ra_rotate_quantize_qkv_noalloc(const ra_problem* p, const v
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_mutex);
-  // First call on this device: look up the array's device address (with the
-  // device current), once.
-  if (g_scratch_dev[dev] == nullptr) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress");
-    g_scratch_dev[dev] = ptr;
-  }
-  char* scratch = static_cast<char*>(g_scratch_dev[dev]);
+  char* scratch = nullptr;
+  if ((e = scratch_address(dev, &scratch)) != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress");
   // Header (cleared error word + this problem's signature) and tables are
   // staged in static host memory and copied in stream order; the pageable
   // copy is staged by the runtime before cudaMemcpyAsync returns, so the
@@ -97,11 +104,52 @@ extern "C" ra_status ra_rotate_quantize_qkv_noalloc(const ra_problem* p, const v
   std::memcpy(g_stage, &hdr, sizeof(hdr));
   ra::build_coef_tables(p, P, reinterpret_cast<float*>(g_stage + L.tables));
   e = cudaMemcpyAsync(scratch, g_stage, L.vamax, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_err(e, "scratch upload");
+  if (e != cudaSuccess) {
+    g_scratch_dev[dev] = nullptr;   // looked up afresh next time (e.g. after a device reset)
+    return cuda_err(e, "scratch upload");
+  }
   // The V amax part is zeroed inside launch_prologue before it accumulates.
   e = ra::launch_prologue(P, static_cast<const __half*>(q), static_cast<const __half*>(k),
                           static_cast<const __half*>(v), out->q4, out->k4, out->v4t, out->sq, out->sk, out->sv,
                           out->vsum, scratch, s);
-  if (e != cudaSuccess) return cuda_err(e, "prologue launch");
+  if (e != cudaSuccess) {
+    g_scratch_dev[dev] = nullptr;
+    return cuda_err(e, "prologue launch");
+  }
   return RA_OK;
+}
+
+extern "C" ra_status ra_noalloc_check_device_error(ra_stream stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_err(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    ra::set_error_detail("device ordinal beyond the per-device table");
+    return RA_ERR_UNSUPPORTED;
+  }
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_err(e, "stream synchronize");
+  char* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if ((e = scratch_address(dev, &scratch)) != cudaSuccess) return cuda_err(e, "cudaGetSymbolAddress");
+  }
+  // the error word is the first member of the scratch's header, as in a
+  // workspace; read it, and clear it when set
+  ra::DeviceErr err{};
+  e = cudaMemcpy(&err, scratch, sizeof(err), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_err(e, "error word read");
+  if (err.word == 0) return RA_OK;
+  e = cudaMemset(scratch, 0, sizeof(err));
+  if (e != cudaSuccess) return cuda_err(e, "error word clear");
+  char msg[160];
+  if (err.word & ra::DEVERR_WORKSPACE) {
+    snprintf(msg, sizeof(msg), "fixed scratch holds another problem's tables: overlapping calls? (site 0x%x)",
+             err.site);
+    ra::set_error_detail(msg);
+    return RA_ERR_WORKSPACE;
+  }
+  snprintf(msg, sizeof(msg), "device-side check in the prologue (site 0x%x)", err.site);
+  ra::set_error_detail(msg);
+  return (err.word & ra::DEVERR_BOUNDS) ? RA_ERR_DEVICE_BOUNDS : RA_ERR_DEVICE_TIMEOUT;
 }

@@ -67,6 +67,7 @@ def test_noalloc_matches_workspace_entry_point(dev):
         buf = torch.full((api.qkv4_bytes(p),), 0x5A, dtype=torch.uint8, device=dev)
         qkv4 = api.qkv4_bind(p, buf)
         api.rotate_quantize_qkv_noalloc(p, q, k, v, qkv4)
+        api.noalloc_check_device_error()            # the scratch's error word is clear
         got = snapshot(buf, qkv4, cfg)
         for f in FIELDS:
             assert np.array_equal(got[f], want[f]), (name, f)
@@ -76,6 +77,28 @@ def test_noalloc_matches_workspace_entry_point(dev):
         api.int4_attention_fwd(p, qkv4, o, ref.workspace)
         ref.check()
         assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16)), name
+
+
+def test_noalloc_on_a_side_stream(dev):
+    # the same call enqueued on a non-default stream: same bytes, clear error word
+    cfg = synth.CONFIGS["tiny"]
+    q, k, v = (torch.from_numpy(t).to(dev) for t in synth.make_qkv(cfg))
+    ref = api.RotateAttention(cfg, dev, fp16_path=False)
+    ref.rotate_quantize(q, k, v)
+    ref.check()
+    want = snapshot(ref.qkv4_buf, ref.qkv4, cfg)
+    p = api.problem(cfg)
+    buf = torch.full((api.qkv4_bytes(p),), 0xA5, dtype=torch.uint8, device=dev)
+    qkv4 = api.qkv4_bind(p, buf)
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        api.rotate_quantize_qkv_noalloc(p, q, k, v, qkv4, stream=side)
+        api.noalloc_check_device_error(stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    got = snapshot(buf, qkv4, cfg)
+    for f in FIELDS:
+        assert np.array_equal(got[f], want[f]), f
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(dev):
