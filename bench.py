@@ -7,7 +7,13 @@ ra_int4_attention_fwd, inputs resident in HBM.  Metric: INT4 attention TOPS
 = 4*N^2*d*H / time.  Prints one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--config wan|hunyuan|half|tiny] [--schedule]
+                  [--config wan|hunyuan|half|tiny|wan_flat] [--schedule]
+
+Besides the step, the line reports: the attention call alone against the
+measured INT8 tensor-core rate (roofline), the prologue against measured HBM
+bandwidth, the FP16 path, the end-to-end host-buffer call, the mixed-precision
+schedule (10 steps x 10 blocks, 48 % INT4; --schedule: the 10 x 40 one), and
+a stress line on flat logits (every exponential computed).
 
 --impl reference times the CPU oracle (the only reference this method has:
 the paper released no kernels) on a bounded sample of the same workload.
@@ -31,7 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from int4_quantized_attention_b200 import synth  # noqa: E402
-from int4_quantized_attention_b200.schedule import BENCH_SCHEDULE  # noqa: E402
+from int4_quantized_attention_b200 import schedule as sched_mod  # noqa: E402
 
 METRIC = "INT4 attention TOPS (4*N^2*d*H/time) and fraction of B200 INT8 tensor peak"
 KERNELS_PER_STEP = 5      # qk_quant, v_amax, v_quant, expand, int4_attn
@@ -201,6 +207,72 @@ def event_time(fn, iters, stream):
     return start.elapsed_time(end) / iters
 
 
+def measure_int8_peak(dev, stream, local):
+    """Dense INT8 tensor-core rate on this GPU, measured now: the library's
+    tcgen05 kind::i8 issue loop (one CTA per SM, the attention kernel's
+    operand layout), as ~50 ms launches (burst, like the attention call) and
+    back to back for about a second (sustained); and cuBLASLt's int8 GEMM
+    (torch._int_mm, 8192^3) for comparison."""
+    import torch
+    from int4_quantized_attention_b200 import api
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    ws = torch.zeros((256,), dtype=torch.uint8, device=dev)
+    out = {"sms": n_sm}
+    with ClockSampler(local) as clk:
+        for n in (128, 256):
+            ops_per_iter = n_sm * 4 * 2 * 128 * n * 32
+            api.measure_mma_i8(n, 2000, n_sm, ws)          # warm-up
+            t = event_time(lambda: api.measure_mma_i8(n, 20000, n_sm, ws), 1, stream)
+            iters = max(1000, int(20000 * 50.0 / max(t, 1e-3)))   # ~50 ms per launch
+            burst = [event_time(lambda: api.measure_mma_i8(n, iters, n_sm, ws), 1, stream) for _ in range(5)]
+            ms_b = statistics.median(burst)
+            reps = max(1, int(1000.0 / ms_b))
+            ms_s = event_time(lambda: api.measure_mma_i8(n, iters, n_sm, ws), reps, stream)
+            out[f"tcgen05_i8_n{n}"] = {"burst_tops": ops_per_iter * iters / (ms_b * 1e-3) / 1e12,
+                                       "sustained_tops": ops_per_iter * iters / (ms_s * 1e-3) / 1e12,
+                                       "launch_ms": ms_b, "sustained_s": reps * ms_s / 1e3}
+        api.check_device_error(ws)
+        try:
+            m = 8192
+            a = torch.randint(-8, 8, (m, m), dtype=torch.int8, device=dev)
+            b = torch.randint(-8, 8, (m, m), dtype=torch.int8, device=dev).t()   # column-major
+            for _ in range(3):
+                torch._int_mm(a, b)
+            ms1 = statistics.median([event_time(lambda: torch._int_mm(a, b), 1, stream) for _ in range(20)])
+            reps = max(1, int(1000.0 / ms1))
+            ms2 = event_time(lambda: torch._int_mm(a, b), reps, stream)
+            out["cublaslt_int8_gemm"] = {"shape": [m, m, m], "burst_tops": 2.0 * m ** 3 / (ms1 * 1e-3) / 1e12,
+                                         "sustained_tops": 2.0 * m ** 3 / (ms2 * 1e-3) / 1e12}
+            del a, b
+        except Exception as e:   # report, do not fail the bench
+            out["cublaslt_int8_gemm"] = {"unavailable": str(e).splitlines()[0][:160]}
+    out["clocks"] = clk.summary()
+    best = max(out["tcgen05_i8_n128"]["burst_tops"], out["tcgen05_i8_n256"]["burst_tops"])
+    best_s = max(out["tcgen05_i8_n128"]["sustained_tops"], out["tcgen05_i8_n256"]["sustained_tops"])
+    out["peak_burst_tops"], out["peak_sustained_tops"] = best, best_s
+    return out
+
+
+def stress_flat(dev, stream, peak, heads=8, steps=5):
+    """Attention call on flat logits (every P code non-zero, no exponential
+    skipped): the Wan shapes with Q/K channels scaled by 0.3, on `heads` heads
+    (heads are independent CTAs, so the rate per call is that of 40)."""
+    import torch
+    from int4_quantized_attention_b200 import api
+    cfg = synth.CONFIGS["wan_flat"].replace(H=heads, name=f"wan_flat-H{heads}")
+    q, k, v = (torch.from_numpy(t).to(dev) for t in synth.make_qkv(cfg))
+    ra = api.RotateAttention(cfg, dev, fp16_path=False)
+    out = torch.empty_like(q)
+    ra.rotate_quantize(q, k, v)
+    for _ in range(3):
+        ra.int4_attention(out)
+    ms = event_time(lambda: ra.int4_attention(out), steps, stream)
+    ra.check()
+    tops = cfg.ops / (ms * 1e-3) / 1e12
+    return {"workload": cfg.name, "H": heads, "N": cfg.N, "int4_attention_ms": ms, "tops": tops,
+            "frac_int8_peak": tops / peak}
+
+
 def our_arm(args, cfg, rank, world):
     import torch
     import torch.distributed as dist
@@ -222,6 +294,14 @@ def our_arm(args, cfg, rank, world):
         ra.rotate_quantize(qd, kd, vd)
         ra.int4_attention(out)
 
+    if args.only_fp16:   # the FP16 path alone (profiler captures)
+        for _ in range(args.warmup):
+            ra.fp16_attention(qd, kd, vd, out)
+        ms = event_time(lambda: ra.fp16_attention(qd, kd, vd, out), args.steps, stream)
+        ra.check()
+        if rank == 0:
+            print(json.dumps({"workload": cfg.name, "fp16_path_ms": ms}), flush=True)
+        return
     for _ in range(args.warmup):
         step()
     ra.check()
@@ -269,17 +349,18 @@ def our_arm(args, cfg, rank, world):
     ra.check()
     ms_e2e = max_over_ranks(ms_e2e, dev)
 
-    sched = None
-    if args.schedule:
-        sched = run_schedule(ra, qd, kd, vd, out, stream)
+    sched = run_schedule(ra, qd, kd, vd, out, stream,
+                         sched_mod.BENCH_SCHEDULE if args.schedule else sched_mod.BENCH_SCHEDULE_SHORT)
+    peak8 = measure_int8_peak(dev, stream, local)
+    stress = None if args.no_stress else stress_flat(dev, stream, peak8["peak_burst_tops"])
 
     if rank != 0:
         return
     ops = cfg.ops
     tops = aggregate_tops(world, ops, ms_step)
     attn_tops = ops / (ms_attn * 1e-3) / 1e12
-    # the attention kernel is timed alone: burst GEMM figure x the int8:bf16 ratio
-    peak_int8 = peaks["bf16"] * INT8_PER_BF16
+    # the attention kernel is timed alone: the burst figure of the INT8 rate probe
+    peak_int8 = peak8["peak_burst_tops"]
     Np = ra.N_pad
     BH = cfg.B * cfg.H
     pro_bytes = (3 * BH * cfg.N * cfg.d * 2            # read q, k, v
@@ -298,10 +379,13 @@ def our_arm(args, cfg, rank, world):
                    "l2": "inputs larger than L2 (q,k,v 2.3 GB; INT8 K/V operand images 0.77 GB per pass)"},
         "roofline": {"kernel": "int4_attn_kernel", "bound": "tensor", "achieved": attn_tops,
                      "peak": peak_int8, "unit": "TOPS", "frac": attn_tops / peak_int8, "traffic": profiled_traffic(cfg),
-                     "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} TF/s x 2 (int8:bf16 nominal "
-                                    f"ratio); of the sustained-based {peaks['bf16_sus'] * INT8_PER_BF16:.0f}: "
-                                    f"{attn_tops / (peaks['bf16_sus'] * INT8_PER_BF16):.3f}; nominal dense int8 4500",
+                     "peak_source": "measured int8: tcgen05 kind::i8 M128xNxK32 issue loop, one CTA per SM, "
+                                    "~50 ms launches (burst), best of N=128/256, this run",
+                     "frac_of_sustained_int8": attn_tops / peak8["peak_sustained_tops"],
+                     "frac_of_bf16_derived": attn_tops / (peaks["bf16"] * INT8_PER_BF16),
+                     "frac_of_nominal_4500": attn_tops / 4500.0,
                      "algorithmic_ops_per_launch": ops},
+        "int8_peak": peak8,
         "int4_attention_ms": ms_attn,
         "prologue": {"ms": ms_pro, "algorithmic_bytes": pro_bytes,
                      "achieved_gbs": pro_bytes / (ms_pro * 1e-3) / 1e9,
@@ -323,38 +407,28 @@ def our_arm(args, cfg, rank, world):
                                                                        "cpu_model")},
         "gpu": torch.cuda.get_device_name(dev),
     }
-    if sched is not None:
-        line["schedule"] = sched
+    line["schedule"] = sched
+    if stress is not None:
+        line["stress_flat_logits"] = stress
     print(json.dumps(line), flush=True)
 
 
-def run_schedule(ra, qd, kd, vd, out, stream):
+def run_schedule(ra, qd, kd, vd, out, stream, schedule):
     """Mixed-precision schedule: per (step, block) the FP16 or the INT4 path,
-    each call timed with events; compared with all-FP16."""
-    import torch
-    kinds = [kind for _, _, kind in BENCH_SCHEDULE.calls()]
-    per = {"int4": [], "fp16": []}
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in kinds]
-    torch.cuda.synchronize()
-    for kind, (a, b) in zip(kinds, evs):
-        a.record(stream)
-        ra.forward(qd, kd, vd, path=kind, out=out)
-        b.record(stream)
-    torch.cuda.synchronize()
-    for kind, (a, b) in zip(kinds, evs):
-        per[kind].append(a.elapsed_time(b))
-    mixed = sum(per["int4"]) + sum(per["fp16"])
-    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in kinds]
-    for a, b in evs2:
-        a.record(stream)
-        ra.forward(qd, kd, vd, path="fp16", out=out)
-        b.record(stream)
-    torch.cuda.synchronize()
-    all16 = sum(a.elapsed_time(b) for a, b in evs2)
+    each call timed with events; compared with the same calls all on FP16."""
+    kinds, ms = sched_mod.run(ra, qd, kd, vd, out, schedule, stream)
+    per = {"int4": [t for kd_, t in zip(kinds, ms) if kd_ == "int4"],
+           "fp16": [t for kd_, t in zip(kinds, ms) if kd_ == "fp16"]}
+    all16 = sched_mod.Schedule(schedule.steps, schedule.blocks, schedule.steps, 0, 0, 0)
+    _, ms16 = sched_mod.run(ra, qd, kd, vd, out, all16, stream)
     ra.check()
-    return {"calls": len(kinds), "int4_fraction": BENCH_SCHEDULE.int4_fraction,
+    mixed = sum(ms)
+    return {"schedule": f"{schedule.steps} steps x {schedule.blocks} blocks, FP16 on the first/last "
+                        f"{schedule.first_steps}/{schedule.last_steps} steps and first/last "
+                        f"{schedule.first_blocks}/{schedule.last_blocks} blocks",
+            "calls": len(kinds), "int4_fraction": schedule.int4_fraction,
             "int4_ms_per_call": statistics.median(per["int4"]), "fp16_ms_per_call": statistics.median(per["fp16"]),
-            "mixed_total_ms": mixed, "all_fp16_total_ms": all16, "speedup_vs_all_fp16": all16 / mixed}
+            "mixed_total_ms": mixed, "all_fp16_total_ms": sum(ms16), "speedup_vs_all_fp16": sum(ms16) / mixed}
 
 
 def main():
@@ -364,7 +438,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="wan", choices=sorted(synth.CONFIGS))
-    ap.add_argument("--schedule", action="store_true", help="also run the 400-call mixed schedule")
+    ap.add_argument("--schedule", action="store_true",
+                    help="run the 400-call mixed schedule (10 steps x 40 blocks) instead of the 100-call one")
+    ap.add_argument("--no-stress", action="store_true", help="skip the flat-logit stress line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
     ap.add_argument("--rot", default=None, choices=["none", "interleaved", "half", "full"],
@@ -374,6 +450,8 @@ def main():
                     help="P quantisation of the INT4 path (range-optimised: the method)")
     ap.add_argument("--chunk-heads", type=int, default=0,
                     help="heads per chunk of the host-buffer pipeline (0: the library's default, B*H/8)")
+    ap.add_argument("--only-fp16", action="store_true",
+                    help="run only warm-up and timed calls of the FP16 path (for profiler captures)")
     ap.add_argument("--only-step", action="store_true",
                     help="run only the warm-up and timed INT4 steps (for profiler captures)")
     args = ap.parse_args()

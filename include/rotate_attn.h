@@ -127,7 +127,12 @@ int ra_seq_pad(const ra_problem *p);
 
 /* Checks a problem: B, H >= 1; d == 128 (else RA_ERR_UNSUPPORTED); grid
  * sizes >= 0 with N >= 1; split entries even, positive, summing to d;
- * rot in ra_rot_mode; theta > 0; every tensor under 2^31 elements per head. */
+ * rot in ra_rot_mode; theta > 0; B*H <= 65535; N <= RA_MAX_TOKENS (else
+ * RA_ERR_UNSUPPORTED).  The INT4 attention accumulates P.V in int32 in
+ * tensor memory: with V codes widened to 16 * code (|.| <= 112) and P weights
+ * code + 8 <= 15 per key, a row's accumulator stays below 112 * 15 * N, which
+ * RA_MAX_TOKENS keeps under 2^31. */
+#define RA_MAX_TOKENS (1 << 20)
 ra_status ra_validate(const ra_problem *p);
 
 /* Bytes of one device buffer that holds all of ra_qkv4 (sub-buffers aligned
@@ -240,16 +245,29 @@ const char *ra_last_error_detail(void);
  * 16 bytes per RoPE table entry, plus a 256-byte header) are rejected with
  * RA_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
  * (no cudaMalloc, cudaFree or allocating library routine); it copies the
- * tables from static host memory with cudaMemcpyAsync on `stream`, then
- * launches the prologue.  The first call on each device also looks up the
- * array's device address (cudaGetSymbolAddress, with that device current);
- * make that first call before any stream capture.  Every call shares the one
- * array and leaves its contents behind; what must start at zero (the error
- * word, the V amax) is cleared by each call.  Calls whose GPU work overlaps
- * (other streams, other host threads) race on the array: serialise them.
+ * tables from static host memory with cudaMemcpyAsync on `stream` (a pageable
+ * copy, so the call returns once the copy is staged, after the work queued
+ * before it on `stream`), then launches the prologue.  The first call on each
+ * device also looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current) and keeps it; make that first call before any stream
+ * capture.  A call that fails drops the kept address, so it is looked up
+ * again after a device reset (cudaDeviceReset invalidates it).  Every call
+ * shares the one array and leaves its contents behind; what must start at
+ * zero (the error word, the V amax) is cleared by each call.  Calls whose GPU
+ * work overlaps (other streams, other host threads) race on the array:
+ * serialise them.  ra_noalloc_check_device_error reports what the kernels
+ * found, a table signature that does not match its problem (the sign of such
+ * a race) included.
  * q, k, v, out: as for ra_rotate_quantize_qkv. */
 ra_status ra_rotate_quantize_qkv_noalloc(const ra_problem *p, const void *q, const void *k, const void *v,
                                          const ra_qkv4 *out, ra_stream stream);
+
+/* The allocation-free counterpart of ra_check_device_error: synchronises
+ * `stream`, reads and clears the error word of the fixed scratch of the
+ * current device.  Returns RA_OK, RA_ERR_WORKSPACE (the tables in the scratch
+ * were not the problem's: overlapping calls), RA_ERR_DEVICE_TIMEOUT,
+ * RA_ERR_DEVICE_BOUNDS or RA_ERR_CUDA.  Allocates nothing. */
+ra_status ra_noalloc_check_device_error(ra_stream stream);
 
 /* ---- test hooks ------------------------------------------------------- */
 
@@ -279,6 +297,29 @@ int ra_host_chunks(const ra_problem *p, int heads_per_chunk, int *sizes, int max
  * and must return RA_ERR_DEVICE_TIMEOUT via ra_check_device_error. */
 void ra_debug_set_wait_timeout_us(uint32_t microseconds);
 ra_status ra_debug_timeout_probe(void *workspace, size_t workspace_bytes, ra_stream stream);
+
+/* The exponent thresholds behind the INT4 attention's exact P decisions:
+ * the code is w = rne(levels * 2^x) for the fp32 exponent x = log2(P), levels
+ * 15 (the method's map, code = w - 8) or 7 (RA_P_SYMMETRIC, code = w); keys
+ * within 2^-19 (relative) of a rounding boundary are decided as
+ * w = k + (x >= T[k]), T[k] the smallest float not below
+ * log2((k + 1/2) / levels).  Writes min(levels, n) thresholds to `out` (host)
+ * and returns levels, or -1 for levels other than 15 and 7. */
+int ra_p_thresholds(int levels, float *out, int n);
+
+/* ---- measurement hook --------------------------------------------------- */
+
+/* Enqueues the INT8 tensor-core rate probe behind the roofline of the INT4
+ * attention (the pages state no peak; this measures the denominator): `ctas`
+ * CTAs of one per SM, each with one thread issuing `iters` x 4 back-to-back
+ * tcgen05.mma.kind::i8 M128 x n x K32 (n = 128 or 256) on shared-memory
+ * operands laid out as the attention kernel's, so one launch performs
+ * ctas * iters * 4 * 2 * 128 * n * 32 integer operations.  The caller times it
+ * with CUDA events on `stream`.  workspace: device, >= 256 bytes (its error
+ * word records a timed-out completion wait; read it with
+ * ra_check_device_error). */
+ra_status ra_measure_mma_i8(int n, int iters, int ctas, void *workspace, size_t workspace_bytes,
+                            ra_stream stream);
 
 #ifdef __cplusplus
 }

@@ -69,8 +69,11 @@ _SIGNATURES = {
     "ra_debug_int4_tile": (ctypes.c_int, [_P, ctypes.POINTER(Qkv4), ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _V, _V, _V, _SZ, _V]),
     "ra_rotate_quantize_qkv_noalloc": (ctypes.c_int, [_P, _V, _V, _V, ctypes.POINTER(Qkv4), _V]),
+    "ra_noalloc_check_device_error": (ctypes.c_int, [_V]),
     "ra_debug_set_wait_timeout_us": (None, [ctypes.c_uint32]),
     "ra_debug_timeout_probe": (ctypes.c_int, [_V, _SZ, _V]),
+    "ra_measure_mma_i8": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _V, _SZ, _V]),
+    "ra_p_thresholds": (ctypes.c_int, [ctypes.c_int, _V, ctypes.c_int]),
 }
 
 
@@ -207,6 +210,11 @@ def rotate_quantize_qkv_noalloc(p: Problem, q, k, v, out: Qkv4, stream=None) -> 
                                                 _stream(stream)))
 
 
+def noalloc_check_device_error(stream=None) -> None:
+    """Read and clear the error word of the allocation-free prologue's scratch."""
+    _check("ra_noalloc_check_device_error", lib().ra_noalloc_check_device_error(_stream(stream)))
+
+
 def check_device_error(workspace, stream=None) -> None:
     _check("ra_check_device_error", lib().ra_check_device_error(_ptr(workspace), _stream(stream)))
 
@@ -232,6 +240,16 @@ def debug_int4_tile(p: Problem, qkv4: Qkv4, bh: int, q_tile: int, kv_tile: int, 
     return s_out, p_out
 
 
+def p_thresholds(levels: int):
+    """The kernel's exponent thresholds for exact P decisions (host copy)."""
+    import numpy as np
+    out = np.zeros((16,), np.float32)
+    n = lib().ra_p_thresholds(levels, out.ctypes.data_as(ctypes.c_void_p), 16)
+    if n < 0:
+        _check("ra_p_thresholds", RA_ERR_INVALID_ARG)
+    return out[:n]
+
+
 def debug_set_wait_timeout_us(microseconds: int) -> None:
     lib().ra_debug_set_wait_timeout_us(microseconds)
 
@@ -239,6 +257,12 @@ def debug_set_wait_timeout_us(microseconds: int) -> None:
 def debug_timeout_probe(workspace, stream=None) -> None:
     _check("ra_debug_timeout_probe",
            lib().ra_debug_timeout_probe(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def measure_mma_i8(n: int, iters: int, ctas: int, workspace, stream=None) -> None:
+    """Enqueue the INT8 tensor-core rate probe (ctas * iters * 4 * 2 * 128 * n * 32 ops)."""
+    _check("ra_measure_mma_i8", lib().ra_measure_mma_i8(n, iters, ctas, _ptr(workspace), workspace.numel(),
+                                                        _stream(stream)))
 
 
 # ---------------------------------------------------------------- convenience

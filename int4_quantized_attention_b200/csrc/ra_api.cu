@@ -79,7 +79,10 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     return fail(RA_ERR_INVALID_ARG, "P quantisation mode %d unknown", p->p_mode);
   if (p->v_rot != 0 && p->v_rot != 1) return fail(RA_ERR_INVALID_ARG, "v_rot must be 0 or 1, not %d", p->v_rot);
   const long long Np = (N + ra::TILE - 1) / ra::TILE * ra::TILE;
-  if (Np * ra::D >= (1ll << 31)) return fail(RA_ERR_UNSUPPORTED, "sequence too long: %lld tokens", N);
+  // The INT4 attention's int32 P.V accumulator holds up to 112 x (sum of P
+  // weights) <= 112 x 15 N: 2^20 tokens keep it inside the int32 range.
+  if (N > ra::MAX_TOKENS)
+    return fail(RA_ERR_UNSUPPORTED, "sequence too long: %lld tokens (at most %d)", N, ra::MAX_TOKENS);
   if ((long long)p->B * p->H > 65535) return fail(RA_ERR_UNSUPPORTED, "B*H > 65535");
   if (out) {
     ra::Prob& P = *out;
@@ -118,6 +121,9 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     P.m_hw = mags[1];
     P.n_tab = toff;
     P.n_tab_all = toff + p->d / 2;
+    P.half4 = 1;
+    for (int s = 0; s < 3; ++s)
+      if ((P.off[s] & 3) || ((p->split[s] / 2) & 3)) P.half4 = 0;
     // what the tables depend on; B and H only size the buffers (checked on the
     // host), so one prepared workspace serves any batch and head count it fits
     uint64_t h = fnv1a(&p->d, sizeof(int) * 5);
@@ -405,6 +411,15 @@ ra_status ra_debug_timeout_probe(void* ws, size_t ws_bytes, ra_stream stream) {
     return fail(RA_ERR_INVALID_ARG, "workspace NULL, misaligned or too small");
   cudaError_t e = ra::launch_timeout_probe(ws, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "timeout probe launch");
+}
+
+ra_status ra_measure_mma_i8(int n, int iters, int ctas, void* ws, size_t ws_bytes, ra_stream stream) {
+  if (n != 128 && n != 256) return fail(RA_ERR_INVALID_ARG, "MMA width %d: 128 or 256", n);
+  if (iters < 1 || ctas < 1) return fail(RA_ERR_INVALID_ARG, "iters and ctas must be >= 1");
+  if (!aligned16(ws) || ws_bytes < sizeof(ra::WsHeader))
+    return fail(RA_ERR_INVALID_ARG, "workspace NULL, misaligned or too small");
+  cudaError_t e = ra::launch_mma_i8_rate(n, iters, ctas, ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "MMA rate launch");
 }
 
 }  // extern "C"

@@ -13,6 +13,7 @@ namespace ra {
 constexpr int D = 128;          // head_dim
 constexpr int QK_BLOCK = 64;    // tokens per Q/K quantisation block
 constexpr int TILE = 128;       // query rows per CTA tile and keys per KV tile
+constexpr int MAX_TOKENS = RA_MAX_TOKENS;   // longest sequence: 1680 N < 2^31 (int32 P.V accumulator)
 
 // Problem with the sizes the kernels need, computed once on the host.
 struct Prob {
@@ -32,6 +33,7 @@ struct Prob {
   uint32_t m_w, m_hw;           // divisors W and Hh * W
   int fastdiv;
   int rot;
+  int half4;                    // every segment and half-segment boundary is a multiple of 4
   int p_mode;                   // ra_p_mode
   int v_rot;                    // 1: Hadamard on V, undone on O (INT4 path)
   uint64_t signature;
@@ -92,6 +94,7 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
                                   cudaStream_t st);
 cudaError_t launch_fp16_attention(const Prob& p, __half* o, void* ws, cudaStream_t st);
 cudaError_t launch_timeout_probe(void* ws, cudaStream_t st);
+cudaError_t launch_mma_i8_rate(int n, int iters, int ctas, void* ws, cudaStream_t st);
 
 // Wall-clock limit (ns) of every bounded device-side wait.
 uint64_t wait_limit();

@@ -58,6 +58,15 @@ def test_validation_codes(lib):
     assert api.validate(prob(rot="blocks_interleaved")) == api.RA_ERR_INVALID_ARG     # no blocks
     skew = tuple(b * 1.01 for b in blocks)                                   # not orthogonal
     assert api.validate(prob(rot="blocks_half", blocks=skew)) == api.RA_ERR_INVALID_ARG
+
+
+def test_longest_sequence_bound(lib):
+    # the int32 P.V accumulator admits N <= 2^20 tokens (112 * 15 * N < 2^31)
+    assert api.validate(prob(F=1, Hh=1, W=1 << 20, n_text=0)) == api.RA_OK
+    assert api.validate(prob(F=1, Hh=1, W=(1 << 20) - 5, n_text=5)) == api.RA_OK
+    assert api.validate(prob(F=1, Hh=1, W=1 << 20, n_text=1)) == api.RA_ERR_UNSUPPORTED
+    assert api.validate(prob(F=16, Hh=256, W=257, n_text=0)) == api.RA_ERR_UNSUPPORTED
+    assert b"at most 1048576" in lib.ra_last_error_detail()
     assert api.validate(prob(theta=0.0)) == api.RA_ERR_INVALID_ARG
     p = prob()
     p.rot = 7
@@ -211,3 +220,18 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
         k += npos[s] * half
     assert k + 64 == len(tab)                 # then the 64 pair-block entries (zero here)
     assert not tab[k:].any()
+
+
+def test_p_decision_thresholds(lib):
+    """The kernel's table behind exact P codes: T[k] is the smallest float not
+    below log2((k + 1/2) / levels) (recomputed here in extended precision), so
+    that x >= T[k] exactly when levels * 2^x >= k + 1/2 for every fp32 x."""
+    ld = np.longdouble
+    for levels in (15, 7):
+        got = api.p_thresholds(levels)
+        assert got.dtype == np.float32 and len(got) == levels
+        for k, t in enumerate(got):
+            exact = np.log2(ld(2 * k + 1) / ld(2 * levels))
+            below = np.nextafter(t, np.float32(-np.inf))
+            assert ld(below) < exact <= ld(t), (levels, k)
+    assert api.lib().ra_p_thresholds(16, None, 0) == -1

@@ -4,12 +4,14 @@ Bars:
   * prologue (INT4 codes, block scales, V channel scales, V column sums):
     bit-exact on every element;
   * int32 S = Q K^T tiles: bit-exact (through the debug export);
-  * P codes: equal except rare +-1 flips where 15 P sits within float
-    rounding of a .5 boundary (the kernel's exp2 is the hardware's);
+  * P codes: bit-exact (both sides decide w = rne(15 2^x) exactly for the
+    same fp32 exponent x; the kernel resolves keys near a rounding boundary
+    from the exponent itself);
   * fp16 output: cosine >= 0.9999 and max |err| <= 2e-2 * max|V| against the
     oracle; the FP16 path: cosine >= 0.9999, max |err| <= 1e-2 * max|V|.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -22,7 +24,6 @@ pytestmark = pytest.mark.gpu
 COS_MIN = 0.9999
 MAXABS_INT4 = 2e-2
 MAXABS_FP16 = 1e-2
-P_FLIP_MAX = 1e-3      # fraction of valid P codes allowed to differ (each by +-1)
 
 
 @pytest.fixture(scope="module")
@@ -132,7 +133,7 @@ def test_int4_S_tiles_bit_exact_and_P_codes(oracle_mod, dev, name):
     ra, _ = run_int4(cfg, dev, q, k, v)
     BH, Np = cfg.B * cfg.H, (cfg.N + 127) // 128 * 128
     nt = Np // 128
-    flips = total = 0
+    total = 0
     cases = {(0, 0, 0), (0, nt - 1, nt - 1), (BH - 1, 0, nt - 1), (BH - 1, nt - 1, 0)}
     refs = {}
     for bh, qt, kt in sorted(cases):
@@ -148,13 +149,9 @@ def test_int4_S_tiles_bit_exact_and_P_codes(oracle_mod, dev, name):
                 continue
             Sr, Pr = oracle_mod.attention_row_debug(cfg, refs[bh], i, kt)
             assert np.array_equal(S[r], Sr), (bh, qt, kt, r)
-            valid = Pr != -128
-            assert np.array_equal(P[r][~valid], Pr[~valid])
-            d = np.abs(P[r][valid].astype(int) - Pr[valid].astype(int))
-            assert d.max(initial=0) <= 1
-            flips += int((d > 0).sum())
-            total += int(valid.sum())
-    assert flips <= P_FLIP_MAX * total + 2, (flips, total)
+            assert np.array_equal(P[r], Pr), (qt, kt, r, np.nonzero(P[r] != Pr)[0][:5])
+            total += int((Pr != -128).sum())
+    assert total > 0
 
 
 @pytest.mark.parametrize("name", ["tiny", "hy_split", "multi_tile", "text_only"])
@@ -213,27 +210,80 @@ def test_unprepared_workspace_is_reported(dev):
 FULL = ["wan", "hunyuan"]
 
 
+def report(name, text):
+    """Append a line to the parity report (RA_PARITY_REPORT, when set)."""
+    path = os.environ.get("RA_PARITY_REPORT")
+    print(text)
+    if path:
+        with open(path, "a") as f:
+            f.write(f"{name}: {text}\n")
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_sampled(oracle_mod, dev, name):
-    """Full-size workload in the benchmark's launch configuration: every
-    prologue element bit-exact; output rows sampled (head 0 and the last head
-    densely, a few rows of every other head, always the ragged last row)."""
+def test_full_size_rows(oracle_mod, dev, name):
+    """Full-size workload in the benchmark's launch configuration.  Every
+    prologue element bit-exact; output rows against the oracle on the sample
+    synth.sample_rows draws: every row of the first and the last head, a
+    seeded 1 % of the rows of every other head, always the ragged last row.
+    Each row on its own: cosine >= 0.9999 and max |err| <= 2e-2 max|V|."""
     cfg = synth.CONFIGS[name]
     q, k, v = synth.make_qkv(cfg)
     ra, o = run_int4(cfg, dev, q, k, v)
     got = ra.unpack()
-    BH, N = cfg.B * cfg.H, cfg.N
-    rng = np.random.default_rng(99)
-    heads = list(range(BH))
-    for bh, ref in check_prologue(oracle_mod, cfg, got, q, k, v, heads):
+    BH = cfg.B * cfg.H
+    sample = synth.sample_rows(cfg)
+    worst_cos, worst_err, nrows = 1.0, 0.0, 0
+    for bh, ref in check_prologue(oracle_mod, cfg, got, q, k, v, range(BH)):
         b, h = divmod(bh, cfg.H)
-        nrows = 96 if bh in (0, BH - 1) else 4
-        rows = np.unique(np.concatenate([rng.choice(N, nrows, replace=False), [0, N - 1]])).astype(np.int64)
+        rows = sample[bh]
         _, out64 = oracle_mod.attention_rows(cfg, ref, rows=rows, want64=True)
         g = o[b, h][rows].astype(np.float64)
-        assert cosine(g, out64) >= COS_MIN, (bh, cosine(g, out64))
-        assert np.abs(g - out64).max() <= MAXABS_INT4 * np.abs(v[b, h].astype(np.float64)).max()
+        num = np.einsum("ij,ij->i", g, out64)
+        den = np.linalg.norm(g, axis=1) * np.linalg.norm(out64, axis=1) + 1e-300
+        row_cos = num / den
+        vmax = np.abs(v[b, h].astype(np.float64)).max()
+        row_err = np.abs(g - out64).max(axis=1) / vmax
+        i = int(np.argmin(row_cos))
+        assert row_cos[i] >= COS_MIN, (bh, int(rows[i]), float(row_cos[i]))
+        assert row_err.max() <= MAXABS_INT4, (bh, int(rows[np.argmax(row_err)]), float(row_err.max()))
+        worst_cos, worst_err = min(worst_cos, float(row_cos.min())), max(worst_err, float(row_err.max()))
+        nrows += len(rows)
+    report(name, f"INT4 rows {nrows} of {BH * cfg.N}: worst row cosine {worst_cos:.8f}, "
+                 f"worst max|err|/max|V| {worst_err:.3e}")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_S_tiles_ragged(oracle_mod, dev, name):
+    """int32 S tiles and P codes bit-exact at full size:
+    the ragged last KV tile (Wan: 80 valid keys; HunyuanVideo: 16, the text
+    tokens) seen from the first, a middle and the ragged last query tile, and a
+    middle KV tile."""
+    cfg = synth.CONFIGS[name]
+    BH = cfg.B * cfg.H
+    cfg1 = cfg.replace(H=1)                     # one head of the recipe is enough for a tile
+    q, k, v = synth.make_qkv(cfg)
+    q, k, v = q[:, :1], k[:, :1], v[:, :1]
+    ra, _ = run_int4(cfg1, dev, q, k, v)
+    Np = (cfg.N + 127) // 128 * 128
+    nt = Np // 128
+    ref = oracle_head(oracle_mod, cfg1, q, k, v, 0, 0)
+    total = 0
+    for qt, kt in [(0, nt - 1), (nt // 2, nt - 1), (nt - 1, nt - 1), (nt - 1, nt // 2)]:
+        S, P = api.debug_int4_tile(ra.p, ra.qkv4, 0, qt, kt, ra.workspace)
+        ra.check()
+        S, P = S.cpu().numpy(), P.cpu().numpy()
+        for r in range(128):
+            i = qt * 128 + r
+            if i >= cfg.N:
+                continue
+            Sr, Pr = oracle_mod.attention_row_debug(cfg1, ref, i, kt)
+            assert np.array_equal(S[r], Sr), (qt, kt, r)
+            assert np.array_equal(P[r], Pr), (qt, kt, r, np.nonzero(P[r] != Pr)[0][:5])
+            total += int((Pr != -128).sum())
+    assert total > 0
+    report(name, f"S tiles and P codes bit-exact ({total} P codes, 4 tiles of head 0, ragged last KV tile)")
 
 
 @pytest.mark.slow
