@@ -64,7 +64,10 @@ namespace ra {
 namespace {
 
 constexpr int NUM_THREADS = 384;
-constexpr int OP_STAGES = 3;   // INT8 K / V^T operand tiles (bulk copies)
+#ifndef RA_OP_STAGES
+#define RA_OP_STAGES 3
+#endif
+constexpr int OP_STAGES = RA_OP_STAGES;   // INT8 K / V^T operand tiles (bulk copies)
 // Register split: launched at LAUNCH_REGS per thread (384 x 168 = 64512);
 // the copy/MMA warpgroup drops to ISSUE_REGS, the two softmax warpgroups
 // rise to SOFTMAX_REGS: 256 x 208 + 128 x 88 = 64512.
@@ -79,23 +82,45 @@ constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
 constexpr int MAGIC_BITS = 0x4B400000;
 constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6)
 
+// Exact P decisions.  The code is w = rne(pscale 2^x) for the fp32 exponent
+// x (pscale = 15, or 7 for the symmetric map).  The fast path takes 2^x from
+// ex2.approx (relative error below 2^-22) and rounds pscale (1 -+ 2^-19) 2^x;
+// where the two roundings agree, no rounding boundary lies within the error
+// of 2^x and both equal the exact code.  Where they differ (a key within
+// 2^-19 of a boundary: rare), the code is decided from the exponent itself:
+// w = w_lo + (x >= T[w_lo]), T[k] the smallest float not below
+// log2((k + 1/2) / pscale), so x >= T[k] exactly when pscale 2^x >= k + 1/2
+// (at the one exact tie, x = -1, this rounds half to even: 7.5 -> 8,
+// 3.5 -> 4).
+#define RA_P_THRESHOLDS_15                                                                             \
+  -0x1.3a0a7ep+2f, -0x1.a934fp+1f, -0x1.4ae00cp+1f, -0x1.0cbd94p+1f, -0x1.bca9c6p+0f, -0x1.728caap+0f, \
+      -0x1.34d9f6p+0f, -0x1p+0f, -0x1.a38c08p-1f, -0x1.51639ap-1f, -0x1.077622p-1f, -0x1.88874cp-2f,   \
+      -0x1.0d58e4p-2f, -0x1.374d64p-3f, -0x1.90aadcp-5f
+#define RA_P_THRESHOLDS_7                                                                              \
+  -0x1.e75766p+1f, -0x1.1c775ap+1f, -0x1.7c44eep+0f, -0x1p+0f, -0x1.465d36p-1f, -0x1.6446p-2f, -0x1.b5ecb6p-4f
+__constant__ float c_pthr[2][16] = {{RA_P_THRESHOLDS_15}, {RA_P_THRESHOLDS_7}};
+const float h_pthr[2][16] = {{RA_P_THRESHOLDS_15}, {RA_P_THRESHOLDS_7}};   // host copy (test hook)
+constexpr float P_REL_WINDOW = 1.9073486328125e-6f;   // 2^-19
+
 // max of three int32 (two compares)
 __device__ __forceinline__ int imax3(int a, int b, int c) { return max(max(a, b), c); }
 
 struct Smem {
   static constexpr uint32_t QA = 0, QB = 16384;   // INT8 Q operand tiles
-  static constexpr uint32_t OP = 32768;           // 3 x 32 KB: INT8 K (+0), V^T (+16 KB)
-  static constexpr uint32_t P = 131072;           // [tile][j % 2] 16 KB u8 P operands, laid out like Q
-  static constexpr uint32_t BAR = 196608;
+  static constexpr uint32_t OP = 32768;           // OP_STAGES x 32 KB: INT8 K (+0), V^T (+16 KB)
+  static constexpr uint32_t P = OP + OP_STAGES * 32768;   // [tile][j % 2] 16 KB u8 P operands, laid out like Q
+  static constexpr uint32_t BAR = P + 65536;
   static constexpr uint32_t BYTES = BAR + 512;
 };
+static_assert(Smem::BYTES + 1024 <= 232448, "shared memory per CTA");
 
 // P_FULL[tile][b] and PV_DONE[tile][b] serve the KV tiles j with j % 2 == b:
 // a softmax warp may store P(j+1) while another still works on P(j).
 enum : int {
-  B_OP_FULL = 0, B_OP_EMPTY = 3, B_QFULL = 6, B_S_FULL = 7, B_S_EMPTY = 9, B_P_FULL = 11, B_PV_DONE = 15,
-  B_DRAIN = 19, NBAR = 21
+  B_OP_FULL = 0, B_OP_EMPTY = OP_STAGES, B_QFULL = 2 * OP_STAGES, B_S_FULL = B_QFULL + 1, B_S_EMPTY = B_S_FULL + 2,
+  B_P_FULL = B_S_EMPTY + 2, B_PV_DONE = B_P_FULL + 4, B_DRAIN = B_PV_DONE + 4, NBAR = B_DRAIN + 2
 };
+static_assert(8 * NBAR + 8 <= 512, "barrier area");
 
 // 4 packed words (32 codes) -> two 16-byte chunks of 16*code, evens then odds
 // per 8-element group.
@@ -233,6 +258,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         // symmetric: pscale 7, code = w.  w = 0 wherever pscale * 2^x <= 1/2,
         // i.e. x <= log2(1 / (2 pscale)) (-4.91 and -3.81): skip_below lies under it.
         const float pscale = P.p_mode == RA_P_SYMMETRIC ? 7.0f : 15.0f;
+        const float plo = pscale * (1.0f - P_REL_WINDOW), phi = pscale * (1.0f + P_REL_WINDOW);   // exact
+        const float* thr = c_pthr[P.p_mode == RA_P_SYMMETRIC ? 1 : 0];
         const float skip_below = P.p_mode == RA_P_SYMMETRIC ? -4.0f : -5.0f;
         const int zp = P.p_mode == RA_P_SYMMETRIC ? 0 : 8;
         const float* skb = a.sk + (size_t)bh * nblk;
@@ -288,8 +315,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           m = m_new;
           const float negm = -m;
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
-          // 64-key half whose largest x is below -5 holds only zero codes.
-          // Skip its exponentials when that is so for every row of the warp.
+          // 64-key half whose largest x is below skip_below holds only zero
+          // codes.  Skip its exponentials when that is so for every row of the warp.
           const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0, c0, negm) < skip_below) != 0,
                                      __all_sync(0xffffffffu, fmaf(mx1, c1, negm) < skip_below) != 0};
           uint32_t L = 0;
@@ -301,16 +328,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               for (int k = 16 * h; k < 16 * h + 16; ++k) pw[k] = 0u;
               continue;
             }
+            const float ch = h ? c1 : c0;
+            uint32_t near = 0;   // non-zero: some key of the half lies within 2^-19 of a rounding boundary
 #pragma unroll
             for (int k = 16 * h; k < 16 * h + 16; k += 2) {   // 8 keys per pair of words: evens, then odds
               uint32_t wb[8];
-              const float ch = h ? c1 : c0;
 #pragma unroll
               for (int e = 0; e < 8; e += 2) {   // x = 256 S c - m, w = rne(pscale 2^x): pairs
                 const int n = 4 * k + e;
-                float x0, x1, w0, w1;
+                float x0, x1, w0, w1, u0, u1;
                 fma2(x0, x1, __int2float_rn((int)s[n]), __int2float_rn((int)s[n + 1]), ch, ch, negm, negm);
-                fma2(w0, w1, pscale, pscale, ex2(x0), ex2(x1), MAGIC, MAGIC);   // low byte = w
+                const float e0 = ex2(x0), e1 = ex2(x1);
+                fma2(w0, w1, plo, plo, e0, e1, MAGIC, MAGIC);   // low byte = rne(pscale (1 - 2^-19) 2^x)
+                fma2(u0, u1, phi, phi, e0, e1, MAGIC, MAGIC);   // low byte = rne(pscale (1 + 2^-19) 2^x)
+                near |= (__float_as_uint(w0) ^ __float_as_uint(u0)) | (__float_as_uint(w1) ^ __float_as_uint(u1));
                 wb[e] = __float_as_uint(w0);
                 wb[e + 1] = __float_as_uint(w1);
               }
@@ -320,6 +351,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               pw[k + 1] = __byte_perm(o13, o57, 0x5410);
               L = __dp4a(pw[k], 0x01010101u, L);
               L = __dp4a(pw[k + 1], 0x01010101u, L);
+            }
+            if (near) {
+              // rare (this thread only): decide the half's keys near a boundary
+              // from the exponent itself, w = w_lo + (x >= T[w_lo])
+#pragma unroll
+              for (int k = 16 * h; k < 16 * h + 16; k += 2) {
+                uint32_t wb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const float x = fmaf(__int2float_rn((int)s[4 * k + e]), ch, negm);
+                  const float ev = ex2(x);
+                  const uint32_t lo = __float_as_uint(fmaf(plo, ev, MAGIC)) & 0xFFu;
+                  const uint32_t hi = __float_as_uint(fmaf(phi, ev, MAGIC)) & 0xFFu;
+                  wb[e] = lo == hi ? lo : lo + (x >= thr[lo] ? 1u : 0u);
+                }
+                const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
+                const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
+                const uint32_t n0w = __byte_perm(e02, e46, 0x5410), n1w = __byte_perm(o13, o57, 0x5410);
+                L = L - __dp4a(pw[k], 0x01010101u, 0u) - __dp4a(pw[k + 1], 0x01010101u, 0u) +
+                    __dp4a(n0w, 0x01010101u, 0u) + __dp4a(n1w, 0x01010101u, 0u);
+                pw[k] = n0w;
+                pw[k + 1] = n1w;
+              }
             }
           }
           if (nvalid < TILE) {   // keys past N leave the normaliser and the operand
@@ -347,15 +401,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           // was issued a whole tile ago) and before P.V(j) adds to it.  The
           // product is taken in fp32 and rounded to an integer by adding
           // 1.5 * 2^23, whose last mantissa bit is worth 1.  |acc| <= 112 l
-          // plus one unit per earlier rescale, so while l < 2^15 both acc and
-          // the product lie below 2^22 and the result is the nearest integer
-          // to acc * alpha.  Larger rows round acc * alpha / 64 (|acc| < 2^28)
-          // and scale it back: at most 64 units off, under 1e-4 s_V in O as
-          // l >= 2^15 there.  A warp with no such row takes the short loop.
+          // plus the rounding of earlier rescales, so while l < 2^15 both acc
+          // and the product lie below 2^22 and the result is the nearest
+          // integer to acc * alpha.  Rows with 2^15 <= l < 2^21 round
+          // acc * alpha / 64 (|acc| < 2^28) and scale it back: at most 64 units
+          // off, under 1e-4 s_V in O as l >= 2^15 there; rows with l >= 2^21
+          // do the same with / 4096 (|acc| < 2^31, the int32 range: the host
+          // admits N <= 2^20, so 112 l <= 1680 N < 2^31), at most 4096 units
+          // off against l >= 2^21.  A warp with no such row takes the short
+          // loop.
           if (__any_sync(0xffffffffu, moved)) {
             if (!(ok = wait_all(B_PV_DONE + 2 * X + ((j - 1) & 1), ((j - 1) >> 1) & 1, 0x4104))) break;
             tc_fence_after();
-            const bool big = l >= 32768.0f;
+            const bool big = l >= 32768.0f, huge = l >= 2097152.0f;
             const bool any_big = __any_sync(0xffffffffu, moved && big);
             uint32_t acc[128];
             tmem_ld128(tO, acc);
@@ -371,8 +429,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
                   acc[e + 1] = __float_as_uint(r1) - (uint32_t)MAGIC_BITS;
                 }
               } else {
-                const float sc = big ? alpha * 0.015625f : alpha;
-                const uint32_t mult = big ? 64u : 1u, add = 0u - (uint32_t)MAGIC_BITS * mult;
+                const float sc = huge ? alpha * 0.000244140625f : (big ? alpha * 0.015625f : alpha);
+                const uint32_t mult = huge ? 4096u : (big ? 64u : 1u), add = 0u - (uint32_t)MAGIC_BITS * mult;
 #pragma unroll
                 for (int e = 0; e < 128; e += 2) {
                   float r0, r1;
@@ -589,3 +647,10 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
 }
 
 }  // namespace ra
+
+extern "C" int ra_p_thresholds(int levels, float* out, int n) {
+  const int k = levels == 15 ? 0 : (levels == 7 ? 1 : -1);
+  if (k < 0) return -1;
+  for (int i = 0; i < levels && i < n; ++i) out[i] = ra::h_pthr[k][i];
+  return levels;
+}

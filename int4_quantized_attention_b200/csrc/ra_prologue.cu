@@ -93,6 +93,17 @@ __device__ __forceinline__ uint32_t int4_nibble_r(float v, float s, float r) {
   return __float_as_uint(t) & 0xFu;
 }
 
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+
+// Eight codes held in the low bytes of w[0..7] (two's complement) -> one
+// word of nibbles, code e in bits 4e .. 4e + 3: the even codes and the odd
+// codes gathered bytewise, then interleaved as low and high nibbles.
+__device__ __forceinline__ uint32_t pack8_low_nibbles(const uint32_t (&w)[8]) {
+  const uint32_t ev = __byte_perm(__byte_perm(w[0], w[2], 0x0040), __byte_perm(w[4], w[6], 0x0040), 0x5410);
+  const uint32_t od = __byte_perm(__byte_perm(w[1], w[3], 0x0040), __byte_perm(w[5], w[7], 0x0040), 0x5410);
+  return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+}
+
 __device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P, uint32_t site) {
   if (hdr->signature == P.signature) return true;
   if (threadIdx.x == 0) report(const_cast<DeviceErr*>(&hdr->err), DEVERR_WORKSPACE, site);
@@ -198,7 +209,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // One CTA = one 64-token block of Q or K of one head (QK_THREADS threads).
 // Thread t holds channels 8*(t%16) .. +7 of rows (t/16) + QK_RSTEP i.
 template <int ROT>
-__global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __half* __restrict__ q,
+__global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF) ? 3 : 4) qk_quant_kernel(Prob P, const __half* __restrict__ q,
                                                        const __half* __restrict__ k, uint8_t* __restrict__ q4,
                                                        uint8_t* __restrict__ k4, float* __restrict__ sq,
                                                        float* __restrict__ sk, const float4* __restrict__ tab,
@@ -232,31 +243,60 @@ __global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __ha
     rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(pt, tab, tp, xf, z[i]);
   }
   if (HALF_PAIRS) {
+    // pair (o_s + i, o_s + i + d_s/2): each thread has its own channel in a
+    // register and reads the partner's value of the same row from shared memory
 #pragma unroll
-    for (int i = 0; i < QK_ROWS; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ys[r0 + QK_RSTEP * i][c0 + e] = z[i][e];
+    for (int i = 0; i < QK_ROWS; ++i) {
+      float4* row = reinterpret_cast<float4*>(&ys[r0 + QK_RSTEP * i][c0]);
+      row[0] = make_float4(z[i][0], z[i][1], z[i][2], z[i][3]);
+      row[1] = make_float4(z[i][4], z[i][5], z[i][6], z[i][7]);
+    }
     __syncthreads();
+    auto pair_rot = [](bool first, float self, float other, const float4& r4) {
+      const float a = first ? self : other, b = first ? other : self;
+      if (ROT == RA_ROT_BLOCKS_HALF)
+        return first ? __fadd_rn(__fmul_rn(r4.x, a), __fmul_rn(r4.y, b))
+                     : __fadd_rn(__fmul_rn(r4.z, a), __fmul_rn(r4.w, b));
+      return first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
+    };
+    if (P.half4) {
+      // every segment and half-segment boundary is a multiple of 4: a group of
+      // 4 channels shares its segment and half, and its partners are 4
+      // consecutive channels (one 16-byte load)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int c = c0 + e;
-      const int s = segment_of(P, c);
-      const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
-      const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
-      const bool first = (c - off) < h;
-      float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ROT == RA_ROT_BLOCKS_HALF)   // block of pair off_s / 2 + i, i = index in the first half
-        r4 = __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)]);
+      for (int q4 = 0; q4 < 2; ++q4) {
+        const int c4 = c0 + 4 * q4;
+        const int s = segment_of(P, c4);
+        const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+        const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
+        const bool first = (c4 - off) < h;
+        const int pc = first ? c4 + h : c4 - h;
+        float4 r4[4];
 #pragma unroll
-      for (int i = 0; i < QK_ROWS; ++i) {
-        const int r = r0 + QK_RSTEP * i;
-        const float a = first ? ys[r][c] : ys[r][c - h];
-        const float b = first ? ys[r][c + h] : ys[r][c];
-        if (ROT == RA_ROT_BLOCKS_HALF)
-          z[i][e] = first ? __fadd_rn(__fmul_rn(r4.x, a), __fmul_rn(r4.y, b))
-                          : __fadd_rn(__fmul_rn(r4.z, a), __fmul_rn(r4.w, b));
-        else
-          z[i][e] = first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
+        for (int e = 0; e < 4; ++e)   // block of pair off_s / 2 + i, i = index in the first half
+          r4[e] = ROT == RA_ROT_BLOCKS_HALF ? __ldg(&tab[P.n_tab + (off >> 1) + (c4 + e - off) - (first ? 0 : h)])
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < QK_ROWS; ++i) {
+          const float4 o = *reinterpret_cast<const float4*>(&ys[r0 + QK_RSTEP * i][pc]);
+          const float other[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) z[i][4 * q4 + e] = pair_rot(first, z[i][4 * q4 + e], other[e], r4[e]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int c = c0 + e;
+        const int s = segment_of(P, c);
+        const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+        const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
+        const bool first = (c - off) < h;
+        const int pc = first ? c + h : c - h;
+        const float4 r4 = ROT == RA_ROT_BLOCKS_HALF ? __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)])
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < QK_ROWS; ++i) z[i][e] = pair_rot(first, z[i][e], ys[r0 + QK_RSTEP * i][pc], r4);
       }
     }
   }
@@ -271,13 +311,27 @@ __global__ void __launch_bounds__(QK_THREADS) qk_quant_kernel(Prob P, const __ha
   amax = block_max(amax, red);
   const float s = __fdiv_rn(amax, 7.0f);
   const float rs = code_recip(s);
+  // codes as in int4_nibble_r, with the closeness to a tie tracked per row
+  // instead of a branch per element: t = z r + 1.5 * 2^23 holds the code in
+  // its low byte (two's complement); a row with any element within 1e-5 of a
+  // tie (or a scale without a usable reciprocal) is redone with the IEEE
+  // quotient
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
-    const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
-    uint32_t packed = 0;
+    uint32_t tb[8];
+    float near = rs == 0.0f ? 1.0f : 0.0f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) packed |= int4_nibble_r(z[i][e], s, rs) << (4 * e);
-    *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = packed;
+    for (int e = 0; e < 8; ++e) {
+      const float t = __fmaf_rn(z[i][e], rs, kMagic);
+      near = fmaxf(near, fabsf(__fmaf_rn(z[i][e], rs, -__fsub_rn(t, kMagic))));
+      tb[e] = __float_as_uint(t);
+    }
+    if (near > 0.49999f) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tb[e] = (uint32_t)int4_code(z[i][e], s);
+    }
+    const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
+    *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = pack8_low_nibbles(tb);
   }
   if (threadIdx.x == 0) scale[blk] = s;
 }
@@ -320,61 +374,119 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
 }
 
-// One CTA = one 64-token block of V of one head: codes with the per-channel
-// scale, transposed packing (channel-major, two tokens per byte) and the
-// block's column sums.
+// Codes of one thread's pair of V rows (tokens i and i+1 of its eight, 8
+// channels each) from t = v r + 1.5 * 2^23 (EXACT: the IEEE quotient
+// instead), folded into the per-channel words (byte i/2 of word e: token i in
+// the low nibble, i+1 in the high one) and the per-channel code sums; `near`
+// tracks the largest distance of v r from its rounding (see int4_nibble_r).
+template <bool EXACT>
+__device__ __forceinline__ void v_code_pair(const float (&f0)[8], const float (&f1)[8], const float (&s)[8],
+                                            const float (&rs)[8], int i, uint32_t (&word)[8], float (&sum)[8],
+                                            float& near) {
+  const uint32_t sel = i == 0 ? 0x3214u : (i == 2 ? 0x3240u : (i == 4 ? 0x3410u : 0x4210u));
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    uint32_t b0, b1;
+    if (EXACT) {
+      const int c0 = int4_code(f0[e], s[e]), c1 = int4_code(f1[e], s[e]);
+      sum[e] += (float)(c0 + c1);
+      b0 = (uint32_t)c0;
+      b1 = (uint32_t)c1;
+    } else {
+      const float t0 = __fmaf_rn(f0[e], rs[e], kMagic), t1 = __fmaf_rn(f1[e], rs[e], kMagic);
+      const float d0 = __fsub_rn(t0, kMagic), d1 = __fsub_rn(t1, kMagic);
+      near = fmax3(near, fabsf(__fmaf_rn(f0[e], rs[e], -d0)), fabsf(__fmaf_rn(f1[e], rs[e], -d1)));
+      sum[e] = __fadd_rn(sum[e], __fadd_rn(d0, d1));   // small integers: exact
+      b0 = __float_as_uint(t0);
+      b1 = __float_as_uint(t1);
+    }
+    word[e] = __byte_perm(word[e], (b0 & 0xFu) | ((b1 << 4) & 0xF0u), sel);
+  }
+}
+
+// All eight rows of one thread's 8-token group: word e = the eight tokens'
+// nibbles of channel 8g + e, sum e = their codes' sum.
+template <bool EXACT>
+__device__ __forceinline__ void v_code_rows(const Prob& P, const __half* __restrict__ x, int n0, int g,
+                                            const float (&s)[8], const float (&rs)[8], uint32_t (&word)[8],
+                                            float (&sum)[8], float& near) {
+  uint4 raw[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = n0 + i;
+    raw[i] = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    word[e] = 0u;
+    sum[e] = 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float f0[8], f1[8];
+    h8_to_f(raw[i], f0);
+    h8_to_f(raw[i + 1], f1);
+    if (P.v_rot) {
+      hadamard128(f0, g);
+      hadamard128(f1, g);
+    }
+    v_code_pair<EXACT>(f0, f1, s, rs, i, word, sum, near);
+  }
+}
+
+// One CTA = one 64-token block of V of one head, 128 threads: thread (g, r)
+// = (t % 16, t / 16) quantises channels 8g .. 8g + 7 of the block's tokens
+// 8r .. 8r + 7 with the per-channel scales and packs, per channel, the eight
+// tokens' codes into one word of the transposed layout; the words and the
+// column sums are exchanged through shared memory so that every thread
+// stores one channel's 32 bytes.
 __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
                                                       const uint32_t* __restrict__ vamax,
                                                       uint8_t* __restrict__ v4t, float* __restrict__ sv,
                                                       int32_t* __restrict__ vsum,
                                                       const WsHeader* __restrict__ hdr) {
-  __shared__ int8_t codes[QK_BLOCK][D + 16];
+  __shared__ uint32_t wsm[8][8 * 16 + 16];   // [token group r][16 e + g], rows 16 banks apart
+  __shared__ float part[4][D];               // column sums of the two groups of each warp
   if (!signature_ok(hdr, P, 0x300)) return;
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  const int g = threadIdx.x & 15, r = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
   float s[8], rs[8];
+  float near = 0.0f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
     rs[e] = code_recip(s[e]);
+    if (rs[e] == 0.0f) near = 1.0f;   // no usable reciprocal: IEEE path
   }
+  const int n0 = blk * QK_BLOCK + 8 * r;
+  uint32_t word[8];
+  float sum[8];
+  v_code_rows<false>(P, x, n0, g, s, rs, word, sum, near);
+  // rare: some element near a tie; the whole warp redoes its rows (the
+  // Hadamard of v_rot shuffles across the warp, so the branch must be uniform)
+  if (__any_sync(0xffffffffu, near > 0.49999f)) v_code_rows<true>(P, x, n0, g, s, rs, word, sum, near);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = blk * QK_BLOCK + r0 + 8 * i;
-    float f[8];
-    if (n < P.N) {
-      h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
-    } else {
+  for (int e = 0; e < 8; ++e) {
+    wsm[r][16 * e + g] = word[e];
+    sum[e] = __fadd_rn(sum[e], __shfl_xor_sync(0xffffffffu, sum[e], 16));   // the warp's other group
+  }
+  if ((threadIdx.x & 16) == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-    }
-    if (P.v_rot) hadamard128(f, g);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)   // the nibble, sign-extended
-      codes[r0 + 8 * i][8 * g + e] = (int8_t)((int)(int4_nibble_r(f[e], s[e], rs[e]) << 28) >> 28);
+    for (int e = 0; e < 8; ++e) part[r >> 1][8 * g + e] = sum[e];
   }
   __syncthreads();
-  const int c = threadIdx.x;
+  const int c = threadIdx.x, ce = c & 7, cg = c >> 3;
   uint32_t w[8];
-  int sum = 0;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int code = codes[8 * t + e][c];
-      sum += code;
-      word |= (uint32_t)(code & 0xF) << (4 * e);
-    }
-    w[t] = word;
-  }
+  for (int t = 0; t < 8; ++t) w[t] = wsm[t][16 * ce + cg];
   // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
   uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
                                         (size_t)(blk % 2) * (QK_BLOCK / 2));
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
+  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] =
+      (int)__fadd_rn(__fadd_rn(part[0][c], part[1][c]), __fadd_rn(part[2][c], part[3][c]));
   if (blk == 0) sv[(size_t)bh * D + c] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
 }
 
