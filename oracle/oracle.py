@@ -60,6 +60,8 @@ def lib():
         _lib.orc_p_code_sym.argtypes = [ctypes.c_float]
         _lib.orc_p_weight.restype = ctypes.c_int
         _lib.orc_p_weight.argtypes = [ctypes.c_float, ctypes.c_int]
+        _lib.orc_p_weight_amb.restype = ctypes.c_int
+        _lib.orc_p_weight_amb.argtypes = [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
         _lib.orc_rope_angle.restype = ctypes.c_double
         _lib.orc_seq_len.restype = ctypes.c_int
         _lib.orc_seq_pad.restype = ctypes.c_int
@@ -123,6 +125,13 @@ def p_weight(x: float, levels: int = 15) -> int:
     return lib().orc_p_weight(ctypes.c_float(x), levels)
 
 
+def p_weight_amb(x: float, levels: int = 15):
+    """(weight, ambiguous?) for the fp32 exponent x."""
+    amb = ctypes.c_int(0)
+    w = lib().orc_p_weight_amb(ctypes.c_float(x), levels, ctypes.byref(amb))
+    return w, bool(amb.value)
+
+
 def _quant_mode(cfg, quant_p) -> int:
     """0: exact P; 1: range-optimised P code; 2: symmetric P code."""
     if not quant_p:
@@ -175,31 +184,64 @@ def quantize_head(cfg, q, k, v, rot: Optional[str] = None):
     return dict(qc=qc, qs=qs, kc=kc, ks=ks, vc=vc, sv=sv, colsum=cs)
 
 
+MAX_AMB = 8     # ambiguous keys recorded per row
+
+
 def attention_rows(cfg, qz: dict, rows=None, tile: int = 128, quant_p: bool = True,
-                   want64: bool = False):
-    """INT4 attention output rows of one head from the prologue outputs `qz`."""
+                   want64: bool = False, ambiguous: bool = False):
+    """INT4 attention output rows of one head from the prologue outputs `qz`.
+    With ambiguous=True also returns, per row, the number of keys whose P
+    code is ambiguous (either rounding is a correct fp32 decision) and the
+    first MAX_AMB of them."""
     if quant_p and tile % 64:
         raise ValueError("the zero-point column sums need tiles that are whole 64-token blocks")
     rows = np.arange(cfg.N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
     out = np.empty((len(rows), cfg.d), np.float16)
     out64 = np.empty((len(rows), cfg.d), np.float64) if want64 else None
+    cnt = np.zeros((len(rows),), np.int32) if ambiguous else None
+    keys = np.full((len(rows), MAX_AMB), -1, np.int32) if ambiguous else None
     lib().orc_attention_rows(ctypes.byref(problem(cfg)), _ptr(rows), len(rows), tile, _quant_mode(cfg, quant_p),
                              _ptr(qz["qc"]), _ptr(qz["qs"]), _ptr(qz["kc"]), _ptr(qz["ks"]),
                              _ptr(qz["vc"]), _ptr(qz["sv"]), _ptr(qz["colsum"]), _ptr(out),
-                             _ptr(out64) if want64 else None)
-    return (out, out64) if want64 else out
+                             _ptr(out64) if want64 else None, _ptr(cnt) if ambiguous else None,
+                             _ptr(keys) if ambiguous else None, MAX_AMB)
+    res = (out, out64) if want64 else out
+    return (res, cnt, keys) if ambiguous else res
 
 
-def attention_row_debug(cfg, qz: dict, i: int, tile_index: int, tile: int = 128):
-    """S (int32) and P codes (int8; -128 past N) of one row for one KV tile."""
+def attention_row_debug(cfg, qz: dict, i: int, tile_index: int, tile: int = 128, with_ambiguous: bool = False):
+    """S (int32) and P codes (int8; -128 past N) of one row for one KV tile;
+    with_ambiguous=True adds a mask of the tile's keys whose P code is
+    ambiguous (either neighbouring code is a correct fp32 decision)."""
     S = np.zeros((tile,), np.int32)
     P = np.zeros((tile,), np.int8)
     o = np.empty((cfg.d,), np.float16)
+    amb = np.full((4096,), -1, np.int32)
+    cnt = ctypes.c_int32(0)
     lib().orc_attention_row(ctypes.byref(problem(cfg)), i, tile, _quant_mode(cfg, True),
                             _ptr(qz["qc"]), _ptr(qz["qs"]), _ptr(qz["kc"]), _ptr(qz["ks"]),
                             _ptr(qz["vc"]), _ptr(qz["sv"]), _ptr(qz["colsum"]), _ptr(o), None,
-                            tile_index, _ptr(S), _ptr(P))
-    return S, P
+                            tile_index, _ptr(S), _ptr(P), _ptr(amb), len(amb), ctypes.byref(cnt), None, 0)
+    if not with_ambiguous:
+        return S, P
+    keys = amb[:min(cnt.value, len(amb))]
+    in_tile = keys[(keys >= tile_index * tile) & (keys < tile_index * tile + tile)] - tile_index * tile
+    mask = np.zeros((tile,), bool)
+    mask[in_tile] = True
+    return S, P, mask
+
+
+def attention_row_flipped(cfg, qz: dict, i: int, flip, tile: int = 128):
+    """Float64 output row i with the ambiguous keys in `flip` decided the
+    other way (one of the other correct results)."""
+    flip = np.ascontiguousarray(flip, np.int32)
+    o = np.empty((cfg.d,), np.float16)
+    o64 = np.empty((cfg.d,), np.float64)
+    lib().orc_attention_row(ctypes.byref(problem(cfg)), i, tile, _quant_mode(cfg, True),
+                            _ptr(qz["qc"]), _ptr(qz["qs"]), _ptr(qz["kc"]), _ptr(qz["ks"]),
+                            _ptr(qz["vc"]), _ptr(qz["sv"]), _ptr(qz["colsum"]), _ptr(o), _ptr(o64),
+                            -1, None, None, None, 0, None, _ptr(flip) if len(flip) else None, len(flip))
+    return o64
 
 
 def softmax_attention_rows(cfg, q: np.ndarray, k: np.ndarray, v: np.ndarray, rows=None) -> np.ndarray:

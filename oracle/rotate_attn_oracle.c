@@ -353,6 +353,31 @@ int orc_p_code_sym(float P) { return (int)nearbyintf(7.0f * P); }
  * 15 * 2^-1 = 7.5 exactly and the round-half-to-even rint gives 8). */
 int orc_p_weight(float x, int levels) { return (int)rint((double)levels * exp2((double)x)); }
 
+/* READING (several correct results): a P code is decided on hardware from an
+ * approximate 2^x with relative error at most ORC_EX2_REL (measured on the
+ * GPU and bounded there by a test).  Where levels * 2^x lies within that
+ * relative distance of a half-integer, either neighbouring weight is a
+ * correct fp32 decision: orc_p_weight_amb returns the exact weight and sets
+ * *amb; the alternative is the other neighbour of that half-integer. */
+#define ORC_EX2_REL 9.5367431640625e-07   /* 2^-20 */
+int orc_p_weight_amb(float x, int levels, int *amb)
+{
+    double v = (double)levels * exp2((double)x);
+    double h = floor(v) + 0.5;               /* nearest half-integer above floor */
+    double dist = fabs(v - h);
+    if (fabs(v - (h - 1.0)) < dist) dist = fabs(v - (h - 1.0));
+    *amb = dist <= v * ORC_EX2_REL;
+    return (int)rint(v);
+}
+
+/* The other weight of an ambiguous key: the neighbour across the half-integer
+ * next to levels * 2^x. */
+static int p_weight_other(float x, int levels, int w)
+{
+    double v = (double)levels * exp2((double)x);
+    return v >= (double)w ? w + 1 : w - 1;
+}
+
 /* One query row i of the INT4 attention (one head), T_kv = `tile` keys per
  * step of the online softmax (128 for the method as built).
  *
@@ -378,12 +403,15 @@ int orc_p_weight(float x, int levels) { return (int)rint((double)levels * exp2((
  * checking the loop against two-pass softmax attention.
  * Optional outputs: o64 [d] (float64 before the fp16 rounding); for tile
  * index dbg_tile >= 0, dbg_S [tile] and dbg_P [tile] (S and P codes of that
- * tile, -128 where the key is past N).
+ * tile, -128 where the key is past N); amb [max_amb] and n_amb: the keys
+ * whose P code is ambiguous (orc_p_weight_amb).  flip [n_flip]: ambiguous
+ * keys to decide the other way (to form the other correct results).
  * colsum: [N_pad/64][d] per-64-block column sums of the V codes. */
 void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
                        const int8_t *qc, const float *qs, const int8_t *kc, const float *ks,
                        const int8_t *vc, const float *sv, const int32_t *colsum,
-                       f16 *o, double *o64, int dbg_tile, int32_t *dbg_S, int8_t *dbg_P)
+                       f16 *o, double *o64, int dbg_tile, int32_t *dbg_S, int8_t *dbg_P,
+                       int32_t *amb, int max_amb, int32_t *n_amb, const int32_t *flip, int n_flip)
 {
     int N = orc_seq_len(p), d = p->d;
     const float inv_sqrt_d = (float)(1.0 / sqrt((double)d));
@@ -428,9 +456,18 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
             int64_t pvi[512] = {0};
             int64_t Li = 0;
             const int zp = quant_p == 2 ? 0 : 8;
+            const int levels = quant_p == 2 ? 7 : 15;
             for (int n = n0; n < n1; ++n) {
                 float x = fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m_new);
-                int code = quant_p == 2 ? orc_p_weight(x, 7) : orc_p_weight(x, 15) - 8;
+                int is_amb = 0;
+                int w = orc_p_weight_amb(x, levels, &is_amb);
+                if (is_amb) {
+                    if (n_amb && *n_amb < max_amb && amb) amb[*n_amb] = n;
+                    if (n_amb) ++*n_amb;
+                    for (int f = 0; f < n_flip; ++f)
+                        if (flip[f] == n) w = p_weight_other(x, levels, w);
+                }
+                int code = w - (quant_p == 2 ? 0 : 8);
                 Li += code + zp;
                 for (int c = 0; c < d; ++c) pvi[c] += (int64_t)code * vc[(size_t)n * d + c];
                 if (j == dbg_tile && dbg_P) dbg_P[n - n0] = (int8_t)code;
@@ -470,18 +507,25 @@ void orc_attention_row(const orc_problem *p, int i, int tile, int quant_p,
     free(acc); free(S); free(sl); free(pv);
 }
 
-/* Rows `rows[0..nrows)` of one head; out: [nrows][d] fp16, out64 optional. */
+/* Rows `rows[0..nrows)` of one head; out: [nrows][d] fp16, out64 optional.
+ * amb_count [nrows] and amb_keys [nrows][max_amb] (optional): the ambiguous
+ * keys of each row (see orc_p_weight_amb), their number and the first
+ * max_amb of them. */
 void orc_attention_rows(const orc_problem *p, const int64_t *rows, int nrows, int tile, int quant_p,
                         const int8_t *qc, const float *qs, const int8_t *kc, const float *ks,
                         const int8_t *vc, const float *sv, const int32_t *colsum,
-                        f16 *out, double *out64)
+                        f16 *out, double *out64, int32_t *amb_count, int32_t *amb_keys, int max_amb)
 {
     int d = p->d;
     #pragma omp parallel for schedule(dynamic, 4)
-    for (int r = 0; r < nrows; ++r)
+    for (int r = 0; r < nrows; ++r) {
+        int32_t cnt = 0;
         orc_attention_row(p, (int)rows[r], tile, quant_p, qc, qs, kc, ks, vc, sv, colsum,
                           out ? out + (size_t)r * d : NULL, out64 ? out64 + (size_t)r * d : NULL,
-                          -1, NULL, NULL);
+                          -1, NULL, NULL, amb_keys ? amb_keys + (size_t)r * max_amb : NULL, max_amb,
+                          &cnt, NULL, 0);
+        if (amb_count) amb_count[r] = cnt;
+    }
 }
 
 /* Float64 softmax attention of one head on given (already position-encoded)

@@ -41,7 +41,10 @@ MUTANTS = {
     "exponent_drops_max": ("fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m_new)",
                            "fmaf((float)S[n - n0], kq * ks[n / QK_BLOCK], -m)"),
     "rescale_sign_log2": ("exp2((double)m - (double)m_new)", "exp2((double)m_new - (double)m)"),
-    "p_weight_levels_16": ("orc_p_weight(x, 15) - 8", "orc_p_weight(x, 16) - 8"),
+    "p_weight_levels_16": ("const int levels = quant_p == 2 ? 7 : 15;", "const int levels = quant_p == 2 ? 7 : 16;"),
+    "amb_weight_floor": ("    return (int)rint(v);", "    return (int)floor(v);"),
+    "amb_window_absolute": ("*amb = dist <= v * ORC_EX2_REL;", "*amb = dist <= ORC_EX2_REL;"),
+    "flip_same_side": ("return v >= (double)w ? w + 1 : w - 1;", "return v >= (double)w ? w - 1 : w + 1;"),
     "p_weight_floor": ("(int)rint((double)levels * exp2((double)x))", "(int)floor((double)levels * exp2((double)x))"),
 }
 

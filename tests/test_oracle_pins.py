@@ -101,6 +101,66 @@ def test_p_weight_matches_the_p_map(oracle_mod):
                 x = np.nextafter(x, np.float32(np.inf))
 
 
+def test_ambiguous_weights_are_those_near_a_boundary(oracle_mod):
+    """orc_p_weight_amb: the same weight as orc_p_weight, flagged ambiguous
+    exactly where levels * 2^x lies within 2^-20 (relative) of a half-integer:
+    the floats next to every rounding boundary are, exact levels and the
+    zero region are not."""
+    ld = np.longdouble
+    rel = 2.0 ** -20
+    for levels in (15, 7):
+        for k in range(levels):
+            edge = np.log2(ld(2 * k + 1) / ld(2 * levels))
+            x = np.float32(edge)
+            for _ in range(2):
+                x = np.nextafter(x, np.float32(-np.inf))
+            for _ in range(5):
+                w, amb = oracle_mod.p_weight_amb(float(x), levels)
+                assert w == oracle_mod.p_weight(float(x), levels)
+                v = levels * np.exp2(ld(x))
+                assert amb == bool(abs(v - (k + ld(0.5))) <= v * ld(rel)), (levels, k, float(x))
+                assert amb                              # the two floats either side are that close
+                x = np.nextafter(x, np.float32(np.inf))
+        for kk in range(1, levels + 1):                 # exact levels: half a unit from any boundary
+            assert not oracle_mod.p_weight_amb(float(np.float32(math.log2(kk / levels))), levels)[1]
+        assert not oracle_mod.p_weight_amb(-30.0, levels)[1]
+
+
+def test_flipping_an_ambiguous_key(oracle_mod):
+    """A key whose exponent is exactly -1 (15 / 2 = 7.5, the one exact tie) is
+    ambiguous; the oracle's row rounds it to 8 (half to even), the flipped row
+    to 7, and both equal the closed form sum w v / sum w on one tile."""
+    cfg = small_cfg(F=2, Hh=8, W=8, rot="none")                        # N = 128: one tile
+    qc = np.zeros((128, 128), np.int8)
+    qc[:, 0] = 1
+    kc = np.zeros((128, 128), np.int8)
+    kc[5, 0] = 7                                 # the row max, S = 7
+    kc[9, 0] = -1                                # S = -1
+    # scales: c = fl(fl(s_Q K) s_K) = 1/8 exactly with s_Q = 1 and this s_K
+    # (K = fl(log2 e) / fl(sqrt 128)), so x = (S - 7) / 8: -1 for key 9
+    ks = np.full(2, np.float32(0.9802581071853638), np.float32)
+    qz = dict(qc=qc, qs=np.ones(2, np.float32), kc=kc, ks=ks)
+    rng = np.random.default_rng(16)
+    vc = rng.integers(-7, 8, (128, 128)).astype(np.int8)
+    qz.update(vc=vc, sv=np.ones(128, np.float32),
+              colsum=vc.astype(np.int32).reshape(2, 64, 128).sum(axis=1).astype(np.int32))
+    (o, o64), cnt, keys = oracle_mod.attention_rows(cfg, qz, rows=np.array([0]), want64=True, ambiguous=True)
+    assert cnt[0] == 1 and keys[0, 0] == 9
+    S = kc[:, 0].astype(np.float64)
+    w = np.rint(15 * np.exp2((S - 7) / 8))
+    assert w[9] == 8 and w[5] == 15
+    ref = (w @ vc.astype(np.float64)) / w.sum()
+    assert np.allclose(o64[0], ref, rtol=1e-12, atol=1e-12)
+    w2 = w.copy()
+    w2[9] = 7
+    ref2 = (w2 @ vc.astype(np.float64)) / w2.sum()
+    got2 = oracle_mod.attention_row_flipped(cfg, qz, 0, [9])
+    assert np.allclose(got2, ref2, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(got2, ref, rtol=1e-6)
+    _, P, mask = oracle_mod.attention_row_debug(cfg, qz, 0, 0, with_ambiguous=True)
+    assert mask[9] and mask.sum() == 1 and P[9] == 0
+
+
 def test_schedule_golden():
     g = json.load(open(os.path.join(GOLDEN, "schedule.json")))
     for c in g["cases"]:
