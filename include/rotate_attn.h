@@ -298,14 +298,11 @@ int ra_host_chunks(const ra_problem *p, int heads_per_chunk, int *sizes, int max
 void ra_debug_set_wait_timeout_us(uint32_t microseconds);
 ra_status ra_debug_timeout_probe(void *workspace, size_t workspace_bytes, ra_stream stream);
 
-/* The exponent thresholds behind the INT4 attention's exact P decisions:
- * the code is w = rne(levels * 2^x) for the fp32 exponent x = log2(P), levels
- * 15 (the method's map, code = w - 8) or 7 (RA_P_SYMMETRIC, code = w); keys
- * within 2^-19 (relative) of a rounding boundary are decided as
- * w = k + (x >= T[k]), T[k] the smallest float not below
- * log2((k + 1/2) / levels).  Writes min(levels, n) thresholds to `out` (host)
- * and returns levels, or -1 for levels other than 15 and 7. */
-int ra_p_thresholds(int levels, float *out, int n);
+/* y[i] = 2^x[i] as the INT4 attention kernel computes it for the P code
+ * (the hardware ex2.approx, flush-to-zero), for n device floats: a test
+ * measures its relative error against float64, the bound behind the
+ * "ambiguous key" reading of P-code parity. */
+ra_status ra_debug_ex2(const float *x, float *y, int n, ra_stream stream);
 
 /* ---- measurement hook --------------------------------------------------- */
 

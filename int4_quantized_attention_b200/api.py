@@ -73,7 +73,7 @@ _SIGNATURES = {
     "ra_debug_set_wait_timeout_us": (None, [ctypes.c_uint32]),
     "ra_debug_timeout_probe": (ctypes.c_int, [_V, _SZ, _V]),
     "ra_measure_mma_i8": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, _V, _SZ, _V]),
-    "ra_p_thresholds": (ctypes.c_int, [ctypes.c_int, _V, ctypes.c_int]),
+    "ra_debug_ex2": (ctypes.c_int, [_V, _V, ctypes.c_int, _V]),
 }
 
 
@@ -240,14 +240,12 @@ def debug_int4_tile(p: Problem, qkv4: Qkv4, bh: int, q_tile: int, kv_tile: int, 
     return s_out, p_out
 
 
-def p_thresholds(levels: int):
-    """The kernel's exponent thresholds for exact P decisions (host copy)."""
-    import numpy as np
-    out = np.zeros((16,), np.float32)
-    n = lib().ra_p_thresholds(levels, out.ctypes.data_as(ctypes.c_void_p), 16)
-    if n < 0:
-        _check("ra_p_thresholds", RA_ERR_INVALID_ARG)
-    return out[:n]
+def debug_ex2(x, stream=None):
+    """The attention kernel's 2^x (ex2.approx) of a device float32 tensor."""
+    import torch
+    y = torch.empty_like(x)
+    _check("ra_debug_ex2", lib().ra_debug_ex2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def debug_set_wait_timeout_us(microseconds: int) -> None:

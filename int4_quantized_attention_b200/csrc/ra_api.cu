@@ -413,6 +413,13 @@ ra_status ra_debug_timeout_probe(void* ws, size_t ws_bytes, ra_stream stream) {
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "timeout probe launch");
 }
 
+ra_status ra_debug_ex2(const float* x, float* y, int n, ra_stream stream) {
+  if (n < 0 || (n > 0 && (!aligned16(x) || !aligned16(y))))
+    return fail(RA_ERR_INVALID_ARG, "ex2 probe: n < 0 or x, y NULL or misaligned");
+  cudaError_t e = ra::launch_ex2_probe(x, y, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "ex2 probe launch");
+}
+
 ra_status ra_measure_mma_i8(int n, int iters, int ctas, void* ws, size_t ws_bytes, ra_stream stream) {
   if (n != 128 && n != 256) return fail(RA_ERR_INVALID_ARG, "MMA width %d: 128 or 256", n);
   if (iters < 1 || ctas < 1) return fail(RA_ERR_INVALID_ARG, "iters and ctas must be >= 1");

@@ -82,26 +82,6 @@ constexpr float MAGIC = 12582912.0f;                           // 1.5 * 2^23
 constexpr int MAGIC_BITS = 0x4B400000;
 constexpr int S_PAD = -4000000;   // below any 256*S (|256 S| <= 1.6e6)
 
-// Exact P decisions.  The code is w = rne(pscale 2^x) for the fp32 exponent
-// x (pscale = 15, or 7 for the symmetric map).  The fast path takes 2^x from
-// ex2.approx (relative error below 2^-22) and rounds pscale (1 -+ 2^-19) 2^x;
-// where the two roundings agree, no rounding boundary lies within the error
-// of 2^x and both equal the exact code.  Where they differ (a key within
-// 2^-19 of a boundary: rare), the code is decided from the exponent itself:
-// w = w_lo + (x >= T[w_lo]), T[k] the smallest float not below
-// log2((k + 1/2) / pscale), so x >= T[k] exactly when pscale 2^x >= k + 1/2
-// (at the one exact tie, x = -1, this rounds half to even: 7.5 -> 8,
-// 3.5 -> 4).
-#define RA_P_THRESHOLDS_15                                                                             \
-  -0x1.3a0a7ep+2f, -0x1.a934fp+1f, -0x1.4ae00cp+1f, -0x1.0cbd94p+1f, -0x1.bca9c6p+0f, -0x1.728caap+0f, \
-      -0x1.34d9f6p+0f, -0x1p+0f, -0x1.a38c08p-1f, -0x1.51639ap-1f, -0x1.077622p-1f, -0x1.88874cp-2f,   \
-      -0x1.0d58e4p-2f, -0x1.374d64p-3f, -0x1.90aadcp-5f
-#define RA_P_THRESHOLDS_7                                                                              \
-  -0x1.e75766p+1f, -0x1.1c775ap+1f, -0x1.7c44eep+0f, -0x1p+0f, -0x1.465d36p-1f, -0x1.6446p-2f, -0x1.b5ecb6p-4f
-__constant__ float c_pthr[2][16] = {{RA_P_THRESHOLDS_15}, {RA_P_THRESHOLDS_7}};
-const float h_pthr[2][16] = {{RA_P_THRESHOLDS_15}, {RA_P_THRESHOLDS_7}};   // host copy (test hook)
-constexpr float P_REL_WINDOW = 1.9073486328125e-6f;   // 2^-19
-
 // max of three int32 (two compares)
 __device__ __forceinline__ int imax3(int a, int b, int c) { return max(max(a, b), c); }
 
@@ -258,8 +238,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         // symmetric: pscale 7, code = w.  w = 0 wherever pscale * 2^x <= 1/2,
         // i.e. x <= log2(1 / (2 pscale)) (-4.91 and -3.81): skip_below lies under it.
         const float pscale = P.p_mode == RA_P_SYMMETRIC ? 7.0f : 15.0f;
-        const float plo = pscale * (1.0f - P_REL_WINDOW), phi = pscale * (1.0f + P_REL_WINDOW);   // exact
-        const float* thr = c_pthr[P.p_mode == RA_P_SYMMETRIC ? 1 : 0];
         const float skip_below = P.p_mode == RA_P_SYMMETRIC ? -4.0f : -5.0f;
         const int zp = P.p_mode == RA_P_SYMMETRIC ? 0 : 8;
         const float* skb = a.sk + (size_t)bh * nblk;
@@ -315,8 +293,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           m = m_new;
           const float negm = -m;
           // w = 0 exactly wherever 15 * 2^x <= 1/2; x is monotone in S, so a
-          // 64-key half whose largest x is below skip_below holds only zero
-          // codes.  Skip its exponentials when that is so for every row of the warp.
+          // 64-key half whose largest x is below -5 holds only zero codes.
+          // Skip its exponentials when that is so for every row of the warp.
           const bool zero_half[2] = {__all_sync(0xffffffffu, fmaf(mx0, c0, negm) < skip_below) != 0,
                                      __all_sync(0xffffffffu, fmaf(mx1, c1, negm) < skip_below) != 0};
           uint32_t L = 0;
@@ -328,20 +306,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               for (int k = 16 * h; k < 16 * h + 16; ++k) pw[k] = 0u;
               continue;
             }
-            const float ch = h ? c1 : c0;
-            uint32_t near = 0;   // non-zero: some key of the half lies within 2^-19 of a rounding boundary
 #pragma unroll
             for (int k = 16 * h; k < 16 * h + 16; k += 2) {   // 8 keys per pair of words: evens, then odds
               uint32_t wb[8];
+              const float ch = h ? c1 : c0;
 #pragma unroll
               for (int e = 0; e < 8; e += 2) {   // x = 256 S c - m, w = rne(pscale 2^x): pairs
                 const int n = 4 * k + e;
-                float x0, x1, w0, w1, u0, u1;
+                float x0, x1, w0, w1;
                 fma2(x0, x1, __int2float_rn((int)s[n]), __int2float_rn((int)s[n + 1]), ch, ch, negm, negm);
-                const float e0 = ex2(x0), e1 = ex2(x1);
-                fma2(w0, w1, plo, plo, e0, e1, MAGIC, MAGIC);   // low byte = rne(pscale (1 - 2^-19) 2^x)
-                fma2(u0, u1, phi, phi, e0, e1, MAGIC, MAGIC);   // low byte = rne(pscale (1 + 2^-19) 2^x)
-                near |= (__float_as_uint(w0) ^ __float_as_uint(u0)) | (__float_as_uint(w1) ^ __float_as_uint(u1));
+                fma2(w0, w1, pscale, pscale, ex2(x0), ex2(x1), MAGIC, MAGIC);   // low byte = w
                 wb[e] = __float_as_uint(w0);
                 wb[e + 1] = __float_as_uint(w1);
               }
@@ -351,29 +325,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
               pw[k + 1] = __byte_perm(o13, o57, 0x5410);
               L = __dp4a(pw[k], 0x01010101u, L);
               L = __dp4a(pw[k + 1], 0x01010101u, L);
-            }
-            if (near) {
-              // rare (this thread only): decide the half's keys near a boundary
-              // from the exponent itself, w = w_lo + (x >= T[w_lo])
-#pragma unroll
-              for (int k = 16 * h; k < 16 * h + 16; k += 2) {
-                uint32_t wb[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const float x = fmaf(__int2float_rn((int)s[4 * k + e]), ch, negm);
-                  const float ev = ex2(x);
-                  const uint32_t lo = __float_as_uint(fmaf(plo, ev, MAGIC)) & 0xFFu;
-                  const uint32_t hi = __float_as_uint(fmaf(phi, ev, MAGIC)) & 0xFFu;
-                  wb[e] = lo == hi ? lo : lo + (x >= thr[lo] ? 1u : 0u);
-                }
-                const uint32_t e02 = __byte_perm(wb[0], wb[2], 0x0040), e46 = __byte_perm(wb[4], wb[6], 0x0040);
-                const uint32_t o13 = __byte_perm(wb[1], wb[3], 0x0040), o57 = __byte_perm(wb[5], wb[7], 0x0040);
-                const uint32_t n0w = __byte_perm(e02, e46, 0x5410), n1w = __byte_perm(o13, o57, 0x5410);
-                L = L - __dp4a(pw[k], 0x01010101u, 0u) - __dp4a(pw[k + 1], 0x01010101u, 0u) +
-                    __dp4a(n0w, 0x01010101u, 0u) + __dp4a(n1w, 0x01010101u, 0u);
-                pw[k] = n0w;
-                pw[k + 1] = n1w;
-              }
             }
           }
           if (nvalid < TILE) {   // keys past N leave the normaliser and the operand
@@ -647,10 +598,3 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
 }
 
 }  // namespace ra
-
-extern "C" int ra_p_thresholds(int levels, float* out, int n) {
-  const int k = levels == 15 ? 0 : (levels == 7 ? 1 : -1);
-  if (k < 0) return -1;
-  for (int i = 0; i < levels && i < n; ++i) out[i] = ra::h_pthr[k][i];
-  return levels;
-}

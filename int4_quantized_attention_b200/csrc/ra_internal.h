@@ -95,6 +95,7 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
 cudaError_t launch_fp16_attention(const Prob& p, __half* o, void* ws, cudaStream_t st);
 cudaError_t launch_timeout_probe(void* ws, cudaStream_t st);
 cudaError_t launch_mma_i8_rate(int n, int iters, int ctas, void* ws, cudaStream_t st);
+cudaError_t launch_ex2_probe(const float* x, float* y, int n, cudaStream_t st);
 
 // Wall-clock limit (ns) of every bounded device-side wait.
 uint64_t wait_limit();

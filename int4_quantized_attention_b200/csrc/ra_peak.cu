@@ -77,3 +77,21 @@ cudaError_t launch_mma_i8_rate(int n, int iters, int ctas, void* ws, cudaStream_
 }
 
 }  // namespace ra
+
+// ---------------------------------------------------------------- ex2 probe
+// y[i] = the INT4 attention kernel's 2^x (ex2.approx.ftz.f32, ra::ex2) for
+// x[i]: a test measures its relative error against float64, which bounds
+// where the kernel's P code may differ from the exact decision.
+namespace ra {
+namespace {
+__global__ void ex2_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = ex2(x[i]);
+}
+}  // namespace
+
+cudaError_t launch_ex2_probe(const float* x, float* y, int n, cudaStream_t st) {
+  if (n > 0) ex2_probe_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
+}  // namespace ra

@@ -374,119 +374,61 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
 }
 
-// Codes of one thread's pair of V rows (tokens i and i+1 of its eight, 8
-// channels each) from t = v r + 1.5 * 2^23 (EXACT: the IEEE quotient
-// instead), folded into the per-channel words (byte i/2 of word e: token i in
-// the low nibble, i+1 in the high one) and the per-channel code sums; `near`
-// tracks the largest distance of v r from its rounding (see int4_nibble_r).
-template <bool EXACT>
-__device__ __forceinline__ void v_code_pair(const float (&f0)[8], const float (&f1)[8], const float (&s)[8],
-                                            const float (&rs)[8], int i, uint32_t (&word)[8], float (&sum)[8],
-                                            float& near) {
-  const uint32_t sel = i == 0 ? 0x3214u : (i == 2 ? 0x3240u : (i == 4 ? 0x3410u : 0x4210u));
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    uint32_t b0, b1;
-    if (EXACT) {
-      const int c0 = int4_code(f0[e], s[e]), c1 = int4_code(f1[e], s[e]);
-      sum[e] += (float)(c0 + c1);
-      b0 = (uint32_t)c0;
-      b1 = (uint32_t)c1;
-    } else {
-      const float t0 = __fmaf_rn(f0[e], rs[e], kMagic), t1 = __fmaf_rn(f1[e], rs[e], kMagic);
-      const float d0 = __fsub_rn(t0, kMagic), d1 = __fsub_rn(t1, kMagic);
-      near = fmax3(near, fabsf(__fmaf_rn(f0[e], rs[e], -d0)), fabsf(__fmaf_rn(f1[e], rs[e], -d1)));
-      sum[e] = __fadd_rn(sum[e], __fadd_rn(d0, d1));   // small integers: exact
-      b0 = __float_as_uint(t0);
-      b1 = __float_as_uint(t1);
-    }
-    word[e] = __byte_perm(word[e], (b0 & 0xFu) | ((b1 << 4) & 0xF0u), sel);
-  }
-}
-
-// All eight rows of one thread's 8-token group: word e = the eight tokens'
-// nibbles of channel 8g + e, sum e = their codes' sum.
-template <bool EXACT>
-__device__ __forceinline__ void v_code_rows(const Prob& P, const __half* __restrict__ x, int n0, int g,
-                                            const float (&s)[8], const float (&rs)[8], uint32_t (&word)[8],
-                                            float (&sum)[8], float& near) {
-  uint4 raw[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int n = n0 + i;
-    raw[i] = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    word[e] = 0u;
-    sum[e] = 0.0f;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    float f0[8], f1[8];
-    h8_to_f(raw[i], f0);
-    h8_to_f(raw[i + 1], f1);
-    if (P.v_rot) {
-      hadamard128(f0, g);
-      hadamard128(f1, g);
-    }
-    v_code_pair<EXACT>(f0, f1, s, rs, i, word, sum, near);
-  }
-}
-
-// One CTA = one 64-token block of V of one head, 128 threads: thread (g, r)
-// = (t % 16, t / 16) quantises channels 8g .. 8g + 7 of the block's tokens
-// 8r .. 8r + 7 with the per-channel scales and packs, per channel, the eight
-// tokens' codes into one word of the transposed layout; the words and the
-// column sums are exchanged through shared memory so that every thread
-// stores one channel's 32 bytes.
+// One CTA = one 64-token block of V of one head: codes with the per-channel
+// scale, transposed packing (channel-major, two tokens per byte) and the
+// block's column sums.
 __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
                                                       const uint32_t* __restrict__ vamax,
                                                       uint8_t* __restrict__ v4t, float* __restrict__ sv,
                                                       int32_t* __restrict__ vsum,
                                                       const WsHeader* __restrict__ hdr) {
-  __shared__ uint32_t wsm[8][8 * 16 + 16];   // [token group r][16 e + g], rows 16 banks apart
-  __shared__ float part[4][D];               // column sums of the two groups of each warp
+  __shared__ int8_t codes[QK_BLOCK][D + 16];
   if (!signature_ok(hdr, P, 0x300)) return;
   const int blk = blockIdx.x, bh = blockIdx.y;
-  const int g = threadIdx.x & 15, r = threadIdx.x >> 4;
+  const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
   float s[8], rs[8];
-  float near = 0.0f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
     rs[e] = code_recip(s[e]);
-    if (rs[e] == 0.0f) near = 1.0f;   // no usable reciprocal: IEEE path
   }
-  const int n0 = blk * QK_BLOCK + 8 * r;
-  uint32_t word[8];
-  float sum[8];
-  v_code_rows<false>(P, x, n0, g, s, rs, word, sum, near);
-  // rare: some element near a tie; the whole warp redoes its rows (the
-  // Hadamard of v_rot shuffles across the warp, so the branch must be uniform)
-  if (__any_sync(0xffffffffu, near > 0.49999f)) v_code_rows<true>(P, x, n0, g, s, rs, word, sum, near);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    wsm[r][16 * e + g] = word[e];
-    sum[e] = __fadd_rn(sum[e], __shfl_xor_sync(0xffffffffu, sum[e], 16));   // the warp's other group
-  }
-  if ((threadIdx.x & 16) == 0) {
+  for (int i = 0; i < 8; ++i) {
+    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    float f[8];
+    if (n < P.N) {
+      h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
+    } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[r >> 1][8 * g + e] = sum[e];
+      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+    }
+    if (P.v_rot) hadamard128(f, g);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)   // the nibble, sign-extended
+      codes[r0 + 8 * i][8 * g + e] = (int8_t)((int)(int4_nibble_r(f[e], s[e], rs[e]) << 28) >> 28);
   }
   __syncthreads();
-  const int c = threadIdx.x, ce = c & 7, cg = c >> 3;
+  const int c = threadIdx.x;
   uint32_t w[8];
+  int sum = 0;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) w[t] = wsm[t][16 * ce + cg];
+  for (int t = 0; t < 8; ++t) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int code = codes[8 * t + e][c];
+      sum += code;
+      word |= (uint32_t)(code & 0xF) << (4 * e);
+    }
+    w[t] = word;
+  }
   // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
   uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
                                         (size_t)(blk % 2) * (QK_BLOCK / 2));
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] =
-      (int)__fadd_rn(__fadd_rn(part[0][c], part[1][c]), __fadd_rn(part[2][c], part[3][c]));
+  vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
   if (blk == 0) sv[(size_t)bh * D + c] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
 }
 

@@ -220,18 +220,3 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
         k += npos[s] * half
     assert k + 64 == len(tab)                 # then the 64 pair-block entries (zero here)
     assert not tab[k:].any()
-
-
-def test_p_decision_thresholds(lib):
-    """The kernel's table behind exact P codes: T[k] is the smallest float not
-    below log2((k + 1/2) / levels) (recomputed here in extended precision), so
-    that x >= T[k] exactly when levels * 2^x >= k + 1/2 for every fp32 x."""
-    ld = np.longdouble
-    for levels in (15, 7):
-        got = api.p_thresholds(levels)
-        assert got.dtype == np.float32 and len(got) == levels
-        for k, t in enumerate(got):
-            exact = np.log2(ld(2 * k + 1) / ld(2 * levels))
-            below = np.nextafter(t, np.float32(-np.inf))
-            assert ld(below) < exact <= ld(t), (levels, k)
-    assert api.lib().ra_p_thresholds(16, None, 0) == -1

@@ -4,11 +4,13 @@ Bars:
   * prologue (INT4 codes, block scales, V channel scales, V column sums):
     bit-exact on every element;
   * int32 S = Q K^T tiles: bit-exact (through the debug export);
-  * P codes: bit-exact (both sides decide w = rne(15 2^x) exactly for the
-    same fp32 exponent x; the kernel resolves keys near a rounding boundary
-    from the exponent itself);
+  * P codes: bit-exact, except at keys the oracle marks ambiguous (15 2^x
+    within the kernel's 2^x error of a half-integer, for the same fp32
+    exponent x on both sides), where either neighbouring code is correct;
   * fp16 output: cosine >= 0.9999 and max |err| <= 2e-2 * max|V| against the
-    oracle; the FP16 path: cosine >= 0.9999, max |err| <= 1e-2 * max|V|.
+    oracle -- at full size row by row, against the oracle's row or, for a row
+    with ambiguous keys, one of its other correct rows; the FP16 path:
+    cosine >= 0.9999, max |err| <= 1e-2 * max|V|.
 """
 import math
 import os
@@ -24,6 +26,7 @@ pytestmark = pytest.mark.gpu
 COS_MIN = 0.9999
 MAXABS_INT4 = 2e-2
 MAXABS_FP16 = 1e-2
+EX2_REL = 2.0 ** -20      # the oracle's bound on the kernel's 2^x error (ambiguous P codes)
 
 
 @pytest.fixture(scope="module")
@@ -52,6 +55,14 @@ def run_int4(cfg, dev, q, k, v):
     o = ra.int4_attention()
     ra.check()
     return ra, o.cpu().numpy()
+
+
+def check_p_codes(got, want, ambiguous, where):
+    """P codes equal, except at keys the oracle marks ambiguous, where the
+    kernel may hold the other neighbouring code."""
+    diff = got.astype(np.int32) - want.astype(np.int32)
+    assert not np.any(diff[~ambiguous]), (where, np.nonzero(diff * ~ambiguous)[0][:5])
+    assert np.all(np.abs(diff[ambiguous]) <= 1), where
 
 
 def oracle_head(oracle_mod, cfg, q, k, v, b, h):
@@ -147,9 +158,9 @@ def test_int4_S_tiles_bit_exact_and_P_codes(oracle_mod, dev, name):
             i = qt * 128 + r
             if i >= cfg.N:
                 continue
-            Sr, Pr = oracle_mod.attention_row_debug(cfg, refs[bh], i, kt)
+            Sr, Pr, amb = oracle_mod.attention_row_debug(cfg, refs[bh], i, kt, with_ambiguous=True)
             assert np.array_equal(S[r], Sr), (bh, qt, kt, r)
-            assert np.array_equal(P[r], Pr), (qt, kt, r, np.nonzero(P[r] != Pr)[0][:5])
+            check_p_codes(P[r], Pr, amb, (bh, qt, kt, r))
             total += int((Pr != -128).sum())
     assert total > 0
 
@@ -233,24 +244,57 @@ def test_full_size_rows(oracle_mod, dev, name):
     got = ra.unpack()
     BH = cfg.B * cfg.H
     sample = synth.sample_rows(cfg)
-    worst_cos, worst_err, nrows = 1.0, 0.0, 0
+    worst_cos, worst_err, nrows, n_amb_rows, n_amb_keys = 1.0, 0.0, 0, 0, 0
     for bh, ref in check_prologue(oracle_mod, cfg, got, q, k, v, range(BH)):
         b, h = divmod(bh, cfg.H)
         rows = sample[bh]
-        _, out64 = oracle_mod.attention_rows(cfg, ref, rows=rows, want64=True)
+        (_, out64), amb_cnt, amb_keys = oracle_mod.attention_rows(cfg, ref, rows=rows, want64=True, ambiguous=True)
         g = o[b, h][rows].astype(np.float64)
-        num = np.einsum("ij,ij->i", g, out64)
-        den = np.linalg.norm(g, axis=1) * np.linalg.norm(out64, axis=1) + 1e-300
-        row_cos = num / den
         vmax = np.abs(v[b, h].astype(np.float64)).max()
-        row_err = np.abs(g - out64).max(axis=1) / vmax
+        row_cos, row_err = row_metrics(g, out64, vmax)
+        # a row with ambiguous keys may equal one of its other correct results
+        for r in np.nonzero(amb_cnt)[0]:
+            n_amb_rows += 1
+            n_amb_keys += int(amb_cnt[r])
+            assert amb_cnt[r] <= oracle_mod.MAX_AMB, (bh, int(rows[r]), int(amb_cnt[r]))
+            keys = amb_keys[r, :amb_cnt[r]]
+            for mask in range(1, 1 << len(keys)):
+                pick = keys[[(mask >> t) & 1 == 1 for t in range(len(keys))]]
+                alt = oracle_mod.attention_row_flipped(cfg, ref, int(rows[r]), pick)
+                c_alt, e_alt = row_metrics(g[r:r + 1], alt[None, :], vmax)
+                if c_alt[0] > row_cos[r]:
+                    row_cos[r], row_err[r] = c_alt[0], e_alt[0]
         i = int(np.argmin(row_cos))
         assert row_cos[i] >= COS_MIN, (bh, int(rows[i]), float(row_cos[i]))
         assert row_err.max() <= MAXABS_INT4, (bh, int(rows[np.argmax(row_err)]), float(row_err.max()))
         worst_cos, worst_err = min(worst_cos, float(row_cos.min())), max(worst_err, float(row_err.max()))
         nrows += len(rows)
     report(name, f"INT4 rows {nrows} of {BH * cfg.N}: worst row cosine {worst_cos:.8f}, "
-                 f"worst max|err|/max|V| {worst_err:.3e}")
+                 f"worst max|err|/max|V| {worst_err:.3e}; rows with ambiguous P codes {n_amb_rows} "
+                 f"({n_amb_keys} keys)")
+
+
+def row_metrics(g, ref, vmax):
+    """Per-row cosine and max |err| / max|V|."""
+    num = np.einsum("ij,ij->i", g, ref)
+    den = np.linalg.norm(g, axis=1) * np.linalg.norm(ref, axis=1) + 1e-300
+    return num / den, np.abs(g - ref).max(axis=1) / vmax
+
+
+def test_kernel_exp2_error_bound(dev):
+    """The kernel's 2^x (ex2.approx) is within EX2_REL of float64 -- the bound
+    the oracle uses to mark ambiguous P codes -- on every float in [-1, -1/2)
+    and on a dense sweep of [-8, 0] (2^x over [-8, 0] covers every nonzero
+    code)."""
+    xs = [np.float32(-1.0) + np.arange(1 << 23, dtype=np.float32) * np.float32(2.0 ** -24),
+          np.linspace(-8.0, 0.0, 1 << 22, dtype=np.float32)]
+    worst = 0.0
+    for x in xs:
+        y = api.debug_ex2(torch.from_numpy(x).to(dev)).cpu().numpy().astype(np.float64)
+        ref = np.exp2(x.astype(np.float64))
+        worst = max(worst, float(np.max(np.abs(y - ref) / ref)))
+    report("ex2", f"max relative error {worst:.3e} = 2^{math.log2(worst):.2f} (bound {EX2_REL:.3e})")
+    assert worst <= EX2_REL
 
 
 @pytest.mark.slow
@@ -269,7 +313,7 @@ def test_full_size_S_tiles_ragged(oracle_mod, dev, name):
     Np = (cfg.N + 127) // 128 * 128
     nt = Np // 128
     ref = oracle_head(oracle_mod, cfg1, q, k, v, 0, 0)
-    total = 0
+    total = ambiguous = 0
     for qt, kt in [(0, nt - 1), (nt // 2, nt - 1), (nt - 1, nt - 1), (nt - 1, nt // 2)]:
         S, P = api.debug_int4_tile(ra.p, ra.qkv4, 0, qt, kt, ra.workspace)
         ra.check()
@@ -278,12 +322,14 @@ def test_full_size_S_tiles_ragged(oracle_mod, dev, name):
             i = qt * 128 + r
             if i >= cfg.N:
                 continue
-            Sr, Pr = oracle_mod.attention_row_debug(cfg1, ref, i, kt)
+            Sr, Pr, amb = oracle_mod.attention_row_debug(cfg1, ref, i, kt, with_ambiguous=True)
             assert np.array_equal(S[r], Sr), (qt, kt, r)
-            assert np.array_equal(P[r], Pr), (qt, kt, r, np.nonzero(P[r] != Pr)[0][:5])
+            check_p_codes(P[r], Pr, amb, (qt, kt, r))
             total += int((Pr != -128).sum())
+            ambiguous += int(amb.sum())
     assert total > 0
-    report(name, f"S tiles and P codes bit-exact ({total} P codes, 4 tiles of head 0, ragged last KV tile)")
+    report(name, f"S tiles bit-exact; P codes bit-exact ({total} codes, {ambiguous} ambiguous; "
+                 f"4 tiles of head 0, ragged last KV tile)")
 
 
 @pytest.mark.slow
