@@ -129,10 +129,11 @@ int ra_seq_pad(const ra_problem *p);
  * sizes >= 0 with N >= 1; split entries even, positive, summing to d;
  * rot in ra_rot_mode; theta > 0; B*H <= 65535; N <= RA_MAX_TOKENS (else
  * RA_ERR_UNSUPPORTED).  The INT4 attention accumulates P.V in int32 in
- * tensor memory: with V codes widened to 16 * code (|.| <= 112) and P weights
- * code + 8 <= 15 per key, a row's accumulator stays below 112 * 15 * N, which
- * RA_MAX_TOKENS keeps under 2^31. */
-#define RA_MAX_TOKENS (1 << 20)
+ * tensor memory, on top of a fixed offset of 0x4B400000 (1,262,485,504): with
+ * V codes widened to 16 * code (|.| <= 112) and P weights code + 8 <= 15 per
+ * key, a row's sum stays within 112 * 15 * N of the offset, which
+ * RA_MAX_TOKENS keeps inside the int32 range. */
+#define RA_MAX_TOKENS (1 << 19)
 ra_status ra_validate(const ra_problem *p);
 
 /* Bytes of one device buffer that holds all of ra_qkv4 (sub-buffers aligned

@@ -12,7 +12,11 @@ import os
 from typing import Optional
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "librotate_attn.so")
+# RA_LIBRARY=bounds loads the bounds-checked test build instead (the same
+# ABI; every computed device index is checked, violations are reported as
+# RA_ERR_DEVICE_BOUNDS by ra_check_device_error).
+LIB_PATH = os.path.join(PKG, "librotate_attn_bounds.so" if os.environ.get("RA_LIBRARY") == "bounds"
+                        else "librotate_attn.so")
 
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_WORKSPACE, RA_ERR_CUDA, \
     RA_ERR_DEVICE_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(7)

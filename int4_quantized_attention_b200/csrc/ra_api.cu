@@ -79,8 +79,9 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
     return fail(RA_ERR_INVALID_ARG, "P quantisation mode %d unknown", p->p_mode);
   if (p->v_rot != 0 && p->v_rot != 1) return fail(RA_ERR_INVALID_ARG, "v_rot must be 0 or 1, not %d", p->v_rot);
   const long long Np = (N + ra::TILE - 1) / ra::TILE * ra::TILE;
-  // The INT4 attention's int32 P.V accumulator holds up to 112 x (sum of P
-  // weights) <= 112 x 15 N: 2^20 tokens keep it inside the int32 range.
+  // The INT4 attention's int32 P.V accumulator holds the offset 0x4B400000
+  // plus up to 112 x (sum of P weights) <= 112 x 15 N: 2^19 tokens keep it
+  // inside the int32 range.
   if (N > ra::MAX_TOKENS)
     return fail(RA_ERR_UNSUPPORTED, "sequence too long: %lld tokens (at most %d)", N, ra::MAX_TOKENS);
   if ((long long)p->B * p->H > 65535) return fail(RA_ERR_UNSUPPORTED, "B*H > 65535");

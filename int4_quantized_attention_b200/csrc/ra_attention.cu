@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(f16::NUM_THREADS, 1)
         // epilogue: O / l -> fp16 for rows < N; loads are warp-collective
         tc_fence_after();
         const float inv = 1.0f / l;
-        const bool store = row < Pb.N;
+        const bool store = row < Pb.N && in_bounds(bh < Pb.BH, err, 0x2211);
         __half* orow = o + ((size_t)bh * Pb.N + (store ? row : 0)) * D;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -237,14 +237,18 @@ __global__ void __launch_bounds__(f16::NUM_THREADS, 1)
       const uint8_t* src = (isK ? kimg : vimg) + (size_t)bh * nt * 32768;
       const int FULL = isK ? B_KFULL : B_VFULL, EMPTY = isK ? B_KEMPTY : B_VEMPTY;
       const uint32_t base = isK ? Smem::K : Smem::V;
-      if (isK) {
+      // the grid covers the problem exactly: every copy below reads tiles
+      // bh * nt + t with t < nt of an image of BH * nt tiles
+      const bool ok_idx = in_bounds(bh < Pb.BH && qt0 + (hasB ? 2 : 1) <= nt, err, 0x2210);
+      if (!ok_idx) *abort_flag = 1;   // every wait gives up; nothing is copied
+      if (isK && ok_idx) {
         const uint8_t* qsrc = qimg + ((size_t)bh * nt + qt0) * 32768;
         mbar_expect_tx(&bar[B_QFULL], hasB ? 65536u : 32768u);
         bulk_g2s(sm + Smem::QA, qsrc, 32768, &bar[B_QFULL]);
         if (hasB) bulk_g2s(sm + Smem::QB, qsrc + 32768, 32768, &bar[B_QFULL]);
       }
       int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = 0; ok_idx && j < nt; ++j) {
         const int st = j % STAGES;
         if (j >= STAGES &&
             !mbar_wait_abortable(&bar[EMPTY + st], ((j / STAGES) - 1) & 1, abort_flag, limit, err, 0x2201))
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(f16::NUM_THREADS, 1)
         issued = j + 1;
       }
       if (*abort_flag) {   // let every copy still in flight land before the CTA exits
-        if (isK) mbar_wait(&bar[B_QFULL], 0, limit, err, 0x2203);
+        if (isK && ok_idx) mbar_wait(&bar[B_QFULL], 0, limit, err, 0x2203);
         for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
           mbar_wait(&bar[FULL + j % STAGES], (j / STAGES) & 1, limit, err, 0x2204);
       }

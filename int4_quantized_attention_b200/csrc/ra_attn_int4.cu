@@ -137,9 +137,12 @@ __device__ __forceinline__ uint32_t p_word_mask(int k, int nvalid) {
 __global__ void __launch_bounds__(256) expand_kernel(const uint8_t* __restrict__ q4, const uint8_t* __restrict__ k4,
                                                      const uint8_t* __restrict__ v4t, uint8_t* __restrict__ qimg,
                                                      uint8_t* __restrict__ kimg, uint8_t* __restrict__ vimg,
-                                                     size_t units) {
+                                                     size_t units, DeviceErr* err) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= units) return;
+  // units = packed bytes / 16 (4 per 128-byte image row, 512 per 16 KB tile);
+  // the images hold 32 bytes per unit
+  if (!in_bounds((i >> 9) * 16384 + 16384 <= units * 32, err, 0x4001)) return;
   const int which = blockIdx.y;
   const uint8_t* src = which == 0 ? q4 : (which == 1 ? k4 : v4t);
   uint8_t* dst = which == 0 ? qimg : (which == 1 ? kimg : vimg);
@@ -189,6 +192,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
   const bool hasB = qt0 + 1 < n_qt;
   DeviceErr* err = &a.hdr->err;
   const uint64_t limit = a.limit;
+  // the grid covers the problem exactly: every index below derives from qt0
+  // (< n_qt), bh (< BH) and the KV tile j (< nt)
+  if (!in_bounds(qt0 < n_qt && bh < P.BH, err, 0x4010)) return;
 
   if (tid == 0) {
     for (int i = 0; i < OP_STAGES; ++i) {
@@ -233,7 +239,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       bool ok = true;
       {
         const int grow = (qt0 + X) * TILE + (int)row;
-        const float kq = __fmul_rn(a.sq[(size_t)bh * nblk + grow / QK_BLOCK], LOG2E / (SQRT_D * 256.0f));
+        const float kq = in_bounds(grow / QK_BLOCK < nblk, err, 0x4011)
+                             ? __fmul_rn(a.sq[(size_t)bh * nblk + grow / QK_BLOCK], LOG2E / (SQRT_D * 256.0f))
+                             : 0.0f;
         // P map: w = rne(pscale * P); range-optimised: pscale 15, code = w - 8;
         // symmetric: pscale 7, code = w.  w = 0 wherever pscale * 2^x <= 1/2,
         // i.e. x <= log2(1 / (2 pscale)) (-4.91 and -3.81): skip_below lies under it.
@@ -248,9 +256,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         float m = -INFINITY, l = 0.0f;
         bool zbuf0 = false, zbuf1 = false;   // this warp's rows of P buffer 0 / 1 hold zeros
         float skn0 = __ldg(skb), skn1 = __ldg(skb + 1);
+        {   // O starts at MB (the bits of 1.5 * 2^23); the P.V MMAs add integers to it
+          uint32_t mb[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mb[e] = (uint32_t)MAGIC_BITS;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_st32(tO + 32 * c, mb);
+          tmem_wait_st();
+        }
         for (int j = 0; j < nt; ++j) {
           const float sk0 = skn0, sk1 = skn1;
-          if (j + 1 < nt) {   // next tile's K scales, a tile ahead
+          if (j + 1 < nt && in_bounds(2 * j + 3 < nblk, err, 0x4012)) {   // next tile's K scales, a tile ahead
             skn0 = __ldg(skb + 2 * j + 2);
             skn1 = __ldg(skb + 2 * j + 3);
           }
@@ -357,10 +373,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           // integer to acc * alpha.  Rows with 2^15 <= l < 2^21 round
           // acc * alpha / 64 (|acc| < 2^28) and scale it back: at most 64 units
           // off, under 1e-4 s_V in O as l >= 2^15 there; rows with l >= 2^21
-          // do the same with / 4096 (|acc| < 2^31, the int32 range: the host
-          // admits N <= 2^20, so 112 l <= 1680 N < 2^31), at most 4096 units
-          // off against l >= 2^21.  A warp with no such row takes the short
-          // loop.
+          // do the same with / 4096 (the host admits N <= 2^19, so
+          // 112 l <= 1680 N keeps MB + acc inside int32), at most 4096 units
+          // off against l >= 2^21.  The accumulator is kept as MB + acc (MB =
+          // the bits of 1.5 * 2^23, written before the first P.V): a short-path
+          // row reads MB + acc as the float 1.5 * 2^23 + acc and rescales it
+          // with one FMA (within one unit); the other rows subtract MB first.
+          // A warp with no large row takes the short loop.
           if (__any_sync(0xffffffffu, moved)) {
             if (!(ok = wait_all(B_PV_DONE + 2 * X + ((j - 1) & 1), ((j - 1) >> 1) & 1, 0x4104))) break;
             tc_fence_after();
@@ -371,21 +390,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
             tmem_wait_ld();
             if (moved) {
               if (!any_big) {
+                // acc = MB + a with |a| < 2^22: read as a float that is
+                // 1.5 * 2^23 + a, and fma(f, alpha, 1.5 * 2^23 (1 - alpha)) rounded
+                // to an integer is 1.5 * 2^23 + a alpha within one unit
+                const float beta = fmaf(-MAGIC, alpha, MAGIC);
 #pragma unroll
                 for (int e = 0; e < 128; e += 2) {
                   float r0, r1;
-                  fma2(r0, r1, __int2float_rn((int)acc[e]), __int2float_rn((int)acc[e + 1]), alpha, alpha, MAGIC,
-                       MAGIC);
-                  acc[e] = __float_as_uint(r0) - (uint32_t)MAGIC_BITS;
-                  acc[e + 1] = __float_as_uint(r1) - (uint32_t)MAGIC_BITS;
+                  fma2(r0, r1, __uint_as_float(acc[e]), __uint_as_float(acc[e + 1]), alpha, alpha, beta, beta);
+                  acc[e] = __float_as_uint(r0);
+                  acc[e + 1] = __float_as_uint(r1);
                 }
               } else {
                 const float sc = huge ? alpha * 0.000244140625f : (big ? alpha * 0.015625f : alpha);
-                const uint32_t mult = huge ? 4096u : (big ? 64u : 1u), add = 0u - (uint32_t)MAGIC_BITS * mult;
+                const uint32_t mult = huge ? 4096u : (big ? 64u : 1u),
+                               add = (uint32_t)MAGIC_BITS - (uint32_t)MAGIC_BITS * mult;
 #pragma unroll
                 for (int e = 0; e < 128; e += 2) {
                   float r0, r1;
-                  fma2(r0, r1, __int2float_rn((int)acc[e]), __int2float_rn((int)acc[e + 1]), sc, sc, MAGIC, MAGIC);
+                  fma2(r0, r1, __int2float_rn((int)(acc[e] - (uint32_t)MAGIC_BITS)),
+                       __int2float_rn((int)(acc[e + 1] - (uint32_t)MAGIC_BITS)), sc, sc, MAGIC, MAGIC);
                   acc[e] = __float_as_uint(r0) * mult + add;
                   acc[e + 1] = __float_as_uint(r1) * mult + add;
                 }
@@ -416,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
           tc_fence_after();
           const float inv = 1.0f / (16.0f * l);
           const float* svb = a.sv + (size_t)bh * D;
-          const bool store = grow < P.N && !dbg_run;
+          const bool store = grow < P.N && !dbg_run && in_bounds(grow < P.N_pad, err, 0x4013);
           __half* orow = a.o + ((size_t)bh * P.N + (store ? grow : 0)) * D;
           if (P.v_rot) {
             // V was quantised as V H / sqrt(128): the row O' = O H / sqrt(128)
@@ -427,7 +451,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
             for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, acc + 32 * c);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 128; ++e) x[e] = (float)(int)acc[e] * __ldg(svb + e) * inv;
+            for (int e = 0; e < 128; ++e) x[e] = (float)(int)(acc[e] - (uint32_t)MAGIC_BITS) * __ldg(svb + e) * inv;
 #pragma unroll
             for (int h = 1; h < 128; h <<= 1)
 #pragma unroll
@@ -459,8 +483,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
             uint32_t hv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float x0 = (float)(int)acc[2 * e] * __ldg(svb + 16 * c + 2 * e) * inv;
-              const float x1 = (float)(int)acc[2 * e + 1] * __ldg(svb + 16 * c + 2 * e + 1) * inv;
+              const float x0 = (float)(int)(acc[2 * e] - (uint32_t)MAGIC_BITS) * __ldg(svb + 16 * c + 2 * e) * inv;
+              const float x1 =
+                  (float)(int)(acc[2 * e + 1] - (uint32_t)MAGIC_BITS) * __ldg(svb + 16 * c + 2 * e + 1) * inv;
               const __half2 h2 = __floats2half2_rn(x0, x1);
               hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
             }
@@ -480,25 +505,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
     // swizzled, K-major), so every tile is one contiguous 16 KB copy.
     if (lane == 0) {
       const uint8_t* qsrc = a.qimg + ((size_t)bh * nt + qt0) * 16384;
-      mbar_expect_tx(&bar[B_QFULL], hasB ? 32768u : 16384u);
-      bulk_g2s(sm + Smem::QA, qsrc, 16384, &bar[B_QFULL]);
-      if (hasB) bulk_g2s(sm + Smem::QB, qsrc + 16384, 16384, &bar[B_QFULL]);
+      const bool q_ok = in_bounds(qt0 + (hasB ? 2 : 1) <= nt, err, 0x4014);
+      if (!q_ok) *abort_flag = 1;   // every wait gives up; nothing is copied
+      if (q_ok) {
+        mbar_expect_tx(&bar[B_QFULL], hasB ? 32768u : 16384u);
+        bulk_g2s(sm + Smem::QA, qsrc, 16384, &bar[B_QFULL]);
+        if (hasB) bulk_g2s(sm + Smem::QB, qsrc + 16384, 16384, &bar[B_QFULL]);
+      }
       const uint8_t* kb = a.kimg + (size_t)bh * nt * 16384;
       const uint8_t* vb = a.vimg + (size_t)bh * nt * 16384;
       int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      for (int j = 0; q_ok && j < nt; ++j) {
         const int st = j % OP_STAGES;
         if (j >= OP_STAGES && !mbar_wait_abortable(&bar[B_OP_EMPTY + st], ((j / OP_STAGES) - 1) & 1, abort_flag,
                                                    limit, err, 0x4201))
           break;
         uint8_t* dst = sm + Smem::OP + st * 32768;
+        if (!in_bounds(j < nt && st < OP_STAGES, err, 0x4015)) {
+          *abort_flag = 1;
+          break;
+        }
         mbar_expect_tx(&bar[B_OP_FULL + st], 32768u);
         bulk_g2s(dst, kb + (size_t)j * 16384, 16384, &bar[B_OP_FULL + st]);
         bulk_g2s(dst + 16384, vb + (size_t)j * 16384, 16384, &bar[B_OP_FULL + st]);
         issued = j + 1;
       }
       if (*abort_flag) {   // let every copy still in flight land before the CTA exits
-        mbar_wait(&bar[B_QFULL], 0, limit, err, 0x4203);
+        if (q_ok) mbar_wait(&bar[B_QFULL], 0, limit, err, 0x4203);
         for (int j = issued > OP_STAGES ? issued - OP_STAGES : 0; j < issued; ++j)
           mbar_wait(&bar[B_OP_FULL + j % OP_STAGES], (j / OP_STAGES) & 1, limit, err, 0x4204);
       }
@@ -519,7 +552,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       const uint32_t op = smem_u32(sm + Smem::OP);
       const uint32_t tS = tbase + X * 128, tO = tbase + 256 + X * 128;
       auto wait = [&](int b, uint32_t parity, uint32_t site) {
-        return mbar_wait_abortable(&bar[b], parity, abort_flag, limit, err, site);
+        return mbar_spin_abortable(&bar[b], parity, abort_flag, limit, err, site);
       };
       auto issue_S = [&](int j) {   // S_X(j) = 256 Q_X K(j)^T
         const uint32_t kt = op + (j % OP_STAGES) * 32768;
@@ -546,7 +579,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         const uint32_t pa = pbase + (j & 1) * 16384;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_i8(tO, sw128_desc(pa + 32 * kk), sw128_desc(vt + 32 * kk), IDESC_PV, (j > 0) || (kk > 0));
+          umma_i8(tO, sw128_desc(pa + 32 * kk), sw128_desc(vt + 32 * kk), IDESC_PV, 1);   // onto MB
         umma_commit(&bar[B_PV_DONE + 2 * X + (j & 1)]);
         umma_commit(&bar[B_OP_EMPTY + j % OP_STAGES]);
       }
@@ -585,7 +618,8 @@ cudaError_t launch_int4_attention(const Prob& p, const uint8_t* q4, const uint8_
   const size_t plane = (size_t)p.BH * p.N_pad * D;   // bytes of one operand image set
   const size_t units = plane / 32;                   // 16 packed bytes -> 32 image bytes
   expand_kernel<<<dim3((unsigned)((units + 255) / 256), 3), 256, 0, st>>>(q4, k4, v4t, img, img + plane,
-                                                                          img + 2 * plane, units);
+                                                                          img + 2 * plane, units,
+                                                                          &static_cast<WsHeader*>(ws)->err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   KernelArgs a{p, img, img + plane, img + 2 * plane, sq, sk, sv, o, static_cast<WsHeader*>(ws), wait_limit(),

@@ -13,7 +13,7 @@ namespace ra {
 constexpr int D = 128;          // head_dim
 constexpr int QK_BLOCK = 64;    // tokens per Q/K quantisation block
 constexpr int TILE = 128;       // query rows per CTA tile and keys per KV tile
-constexpr int MAX_TOKENS = RA_MAX_TOKENS;   // longest sequence: 1680 N < 2^31 (int32 P.V accumulator)
+constexpr int MAX_TOKENS = RA_MAX_TOKENS;   // longest sequence: 0x4B400000 + 1680 N < 2^31 (P.V accumulator)
 
 // Problem with the sizes the kernels need, computed once on the host.
 struct Prob {

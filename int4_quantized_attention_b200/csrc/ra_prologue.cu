@@ -141,11 +141,12 @@ __device__ __forceinline__ PairTab pair_tab(const Prob& P, int c0) {
 // host (m00, m01, m10, m11).
 template <int FORM>
 __device__ __forceinline__ void rope8(const PairTab& pt, const float4* __restrict__ tab, const TokenPos& tp,
-                                      const float (&x)[8], float (&y)[8]) {
+                                      const float (&x)[8], float (&y)[8], int n_tab, DeviceErr* err) {
 #pragma unroll
   for (int pp = 0; pp < 4; ++pp) {
     const int pos = sel3(pt.axis[pp], tp.p[0], tp.p[1], tp.p[2]);
-    const float4 t = __ldg(&tab[pt.base[pp] + pos * pt.stride[pp]]);
+    const int ti = pt.base[pp] + pos * pt.stride[pp];
+    const float4 t = in_bounds(ti >= 0 && ti < n_tab, err, 0x101) ? __ldg(&tab[ti]) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
     if (FORM == 1) {          // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
       y[2 * pp] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
   constexpr bool HALF_PAIRS = ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF;
   __shared__ float ys[HALF_PAIRS ? QK_BLOCK : 1][HALF_PAIRS ? D + 4 : 1];
   if (!signature_ok(hdr, P, 0x100)) return;
+  DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
   uint8_t* out = (which ? k4 : q4) + (size_t)bh * P.N_pad * (D / 2);
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
-    raw[i] = n < P.N ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
+    raw[i] = n < P.N && in_bounds(bh < P.BH, err, 0x102) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0))
+                                                         : make_uint4(0, 0, 0, 0);
   }
   float z[QK_ROWS][8];
   float amax = 0.0f;
@@ -240,7 +243,8 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
     float xf[8];
     h8_to_f(raw[i], xf);
     const TokenPos tp = token_pos(P, n < P.N ? n : 0);
-    rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(pt, tab, tp, xf, z[i]);
+    rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(pt, tab, tp, xf, z[i], P.n_tab,
+                                                                                      err);
   }
   if (HALF_PAIRS) {
     // pair (o_s + i, o_s + i + d_s/2): each thread has its own channel in a
@@ -274,7 +278,9 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
         float4 r4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)   // block of pair off_s / 2 + i, i = index in the first half
-          r4[e] = ROT == RA_ROT_BLOCKS_HALF ? __ldg(&tab[P.n_tab + (off >> 1) + (c4 + e - off) - (first ? 0 : h)])
+          r4[e] = ROT == RA_ROT_BLOCKS_HALF &&
+                          in_bounds((off >> 1) + (c4 + e - off) - (first ? 0 : h) < D / 2, err, 0x103)
+                      ? __ldg(&tab[P.n_tab + (off >> 1) + (c4 + e - off) - (first ? 0 : h)])
                                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < QK_ROWS; ++i) {
@@ -293,7 +299,9 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
         const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
         const bool first = (c - off) < h;
         const int pc = first ? c + h : c - h;
-        const float4 r4 = ROT == RA_ROT_BLOCKS_HALF ? __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)])
+        const float4 r4 = ROT == RA_ROT_BLOCKS_HALF &&
+                                  in_bounds((off >> 1) + (c - off) - (first ? 0 : h) < D / 2, err, 0x104)
+                              ? __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)])
                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < QK_ROWS; ++i) z[i][e] = pair_rot(first, z[i][e], ys[r0 + QK_RSTEP * i][pc], r4);
@@ -331,9 +339,10 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
       for (int e = 0; e < 8; ++e) tb[e] = (uint32_t)int4_code(z[i][e], s);
     }
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
-    *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = pack8_low_nibbles(tb);
+    if (in_bounds(n < P.N_pad && bh < P.BH, err, 0x105))
+      *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = pack8_low_nibbles(tb);
   }
-  if (threadIdx.x == 0) scale[blk] = s;
+  if (threadIdx.x == 0 && in_bounds(blk < P.N_pad / QK_BLOCK && bh < P.BH, err, 0x106)) scale[blk] = s;
 }
 
 // Per-(head, channel) amax of V over a 256-token chunk, merged with
@@ -343,6 +352,7 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
                                                      const WsHeader* __restrict__ hdr) {
   __shared__ float part[8][D];
   if (!signature_ok(hdr, P, 0x200)) return;
+  DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int chunk = blockIdx.x, bh = blockIdx.y;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
@@ -354,7 +364,7 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   for (int i = 0; i < iters; ++i) {
     const int n = chunk * 256 + r0 + 8 * i;
     float f[8];
-    if (n < P.N) {
+    if (n < P.N && in_bounds(bh < P.BH, err, 0x201)) {
       h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
     } else {
 #pragma unroll
@@ -371,7 +381,7 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   float r = part[0][c];
 #pragma unroll
   for (int i = 1; i < 8; ++i) r = fmaxf(r, part[i][c]);
-  atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
+  if (in_bounds(bh < P.BH, err, 0x202)) atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
 }
 
 // One CTA = one 64-token block of V of one head: codes with the per-channel
@@ -384,6 +394,7 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
                                                       const WsHeader* __restrict__ hdr) {
   __shared__ int8_t codes[QK_BLOCK][D + 16];
   if (!signature_ok(hdr, P, 0x300)) return;
+  DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
@@ -397,7 +408,7 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
   for (int i = 0; i < 8; ++i) {
     const int n = blk * QK_BLOCK + r0 + 8 * i;
     float f[8];
-    if (n < P.N) {
+    if (n < P.N && in_bounds(bh < P.BH, err, 0x301)) {
       h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
     } else {
 #pragma unroll
@@ -426,6 +437,7 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
   // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
   uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
                                         (size_t)(blk % 2) * (QK_BLOCK / 2));
+  if (!in_bounds(bh < P.BH && blk < P.N_pad / QK_BLOCK, err, 0x302)) return;
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
   vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
@@ -442,7 +454,9 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
                                                             const WsHeader* __restrict__ hdr) {
   __shared__ __half tr[QK_BLOCK][D + 8];
   if (!signature_ok(hdr, P, 0x400)) return;
+  DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  if (!in_bounds(bh < P.BH && blk < P.N_pad / QK_BLOCK, err, 0x401)) return;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const int c0 = 8 * g;
   const int nt = P.N_pad / TILE;
@@ -458,7 +472,7 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
       if (n < P.N) {
         float xf[8], y[8];
         h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)), xf);
-        rope8<0>(pair_tab(P, c0), tab, token_pos(P, n), xf, y);
+        rope8<0>(pair_tab(P, c0), tab, token_pos(P, n), xf, y, P.n_tab, err);
         __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);

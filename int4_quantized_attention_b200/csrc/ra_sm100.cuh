@@ -25,6 +25,27 @@ __device__ __forceinline__ void report(DeviceErr* e, uint32_t bit, uint32_t site
   if ((atomicOr(&e->word, bit) & bit) == 0) atomicCAS(&e->site, 0u, site);
 }
 
+// Index self-checks.  The library is also built with RA_BOUNDS_CHECK=1
+// (librotate_attn_bounds.so, a test build standing in for a memory checker):
+// there every computed global-memory index is checked against its buffer
+// before the access, and a violation records DEVERR_BOUNDS with the first
+// site and skips the access.  In the production build the checks compile
+// away.
+#ifndef RA_BOUNDS_CHECK
+#define RA_BOUNDS_CHECK 0
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, DeviceErr* e, uint32_t site) {
+#if RA_BOUNDS_CHECK
+  if (!ok) report(e, DEVERR_BOUNDS, site);
+  return ok;
+#else
+  (void)ok;
+  (void)e;
+  (void)site;
+  return true;
+#endif
+}
+
 // ---------------------------------------------------------------- smem
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -61,12 +61,15 @@ def test_validation_codes(lib):
 
 
 def test_longest_sequence_bound(lib):
-    # the int32 P.V accumulator admits N <= 2^20 tokens (112 * 15 * N < 2^31)
-    assert api.validate(prob(F=1, Hh=1, W=1 << 20, n_text=0)) == api.RA_OK
-    assert api.validate(prob(F=1, Hh=1, W=(1 << 20) - 5, n_text=5)) == api.RA_OK
-    assert api.validate(prob(F=1, Hh=1, W=1 << 20, n_text=1)) == api.RA_ERR_UNSUPPORTED
-    assert api.validate(prob(F=16, Hh=256, W=257, n_text=0)) == api.RA_ERR_UNSUPPORTED
-    assert b"at most 1048576" in lib.ra_last_error_detail()
+    # the int32 P.V accumulator (offset 0x4B400000 plus up to 112 * 15 * N)
+    # admits N <= 2^19 tokens
+    assert 0x4B400000 + 112 * 15 * (1 << 19) < 2 ** 31
+    assert 0x4B400000 + 112 * 15 * ((1 << 19) + 4096) >= 2 ** 31   # the bound is within 1 % of tight
+    assert api.validate(prob(F=1, Hh=1, W=1 << 19, n_text=0)) == api.RA_OK
+    assert api.validate(prob(F=1, Hh=1, W=(1 << 19) - 5, n_text=5)) == api.RA_OK
+    assert api.validate(prob(F=1, Hh=1, W=1 << 19, n_text=1)) == api.RA_ERR_UNSUPPORTED
+    assert api.validate(prob(F=8, Hh=256, W=257, n_text=0)) == api.RA_ERR_UNSUPPORTED
+    assert b"at most 524288" in lib.ra_last_error_detail()
     assert api.validate(prob(theta=0.0)) == api.RA_ERR_INVALID_ARG
     p = prob()
     p.rot = 7

@@ -7,8 +7,10 @@ bits(1.5 * 2^23).  Rows with 2^15 <= l < 2^21 take acc * alpha / 64 the same
 way and multiply back by 64; rows with l >= 2^21 use / 4096.  The claims: the
 short path gives exactly rne(acc * alpha) for |acc| < 2^22; the /64 path is
 within 64 units for |acc| < 2^28; the /4096 path is within 4096 units over
-the accumulator's whole range (|acc| <= 112 l <= 1680 N < 2^31 for N <= 2^20
-tokens, the longest sequence the host accepts).
+the accumulator's whole range (|acc| <= 112 l <= 1680 N for N <= 2^19 tokens,
+the longest sequence the host accepts).  The kernel keeps the accumulator as
+MB + acc (MB = bits of 1.5 * 2^23): short-path rows rescale MB + acc with one
+FMA (within one unit, below), the others subtract MB first.
 
 float32 products are exact in float64, so the FMA is the float64 sum rounded
 once to float32; float32(int) is round-to-nearest like cvt.rn.f32.s32.
@@ -76,7 +78,7 @@ def test_short_path_breaks_past_its_range():
 
 def test_huge_path_error_bound_over_int32():
     rng = np.random.default_rng(14)
-    top = 112 * 15 * (1 << 20)          # largest |acc| of the longest accepted sequence
+    top = 112 * 15 * (1 << 19)          # largest |acc| of the longest accepted sequence
     acc = rng.integers(-top, top + 1, 400000, dtype=np.int64)
     acc[:2] = [top, -top]
     a = alphas(rng, acc.size)
@@ -87,10 +89,10 @@ def test_huge_path_error_bound_over_int32():
 
 def test_accumulator_bound_at_the_longest_sequence():
     # 112 = |16 * 7| (widened V code), 15 = largest P weight: the worst row of
-    # the longest accepted sequence still fits int32, one token more of
-    # weight-15 keys would be within 1680 of the edge
-    n_max = 1 << 20
-    assert 112 * 15 * n_max < (1 << 31)
+    # the longest accepted sequence, on top of the offset MB, still fits int32
+    n_max = 1 << 19
+    assert int(MAGIC_BITS) + 112 * 15 * n_max < (1 << 31)
+    assert int(MAGIC_BITS) - 112 * 15 * n_max > -(1 << 31)
     # the tier thresholds: the exact path needs 112 l < 2^22 for l < 2^15,
     # the /64 path 112 l < 2^28 for l < 2^21
     assert 112 * (1 << 15) < (1 << 22)
