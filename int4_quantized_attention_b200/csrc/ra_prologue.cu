@@ -67,33 +67,65 @@ __device__ __forceinline__ int int4_code(float v, float s) {
   return q > 7 ? 7 : (q < -7 ? -7 : q);
 }
 
-// Reciprocal of a block scale for int4_nibble_r: RN(1 / s), or 0 where it
-// would not be a finite normal number (s == 0, or s so small or so large that
-// 1 / s overflows or is subnormal), which sends every element to int4_code.
+// Reciprocal of a scale for int4_codes8: RN(1 / s), or 0 where it would not
+// be a finite normal number (s == 0, or s so small or so large that 1 / s
+// overflows or is subnormal), which sends the elements to int4_code.
 __device__ __forceinline__ float code_recip(float s) {
   const float r = __fdiv_rn(1.0f, s);
   return (r < 3.0e38f && r > 1.0e-37f) ? r : 0.0f;
 }
 
-// The low nibble of int4_code(v, s) without a division per element, for |v| <= 7 s (1 + 2^-22)
-// (every element of the block whose amax gave s = fl(amax / 7)).  With
-// r = RN(1 / s), |v r - v / s| <= |v| 2^-24 / s <= 7.0 * 2^-24 and
-// |fl(v / s) - v / s| <= 2^-22, so v r is within 6.6e-7 of fl(v / s): the two
-// round to the same integer unless v r lies within that of a half-integer.
-// t = v r + 1.5 * 2^23 rounded once is that integer in the low mantissa bits
-// (exact: |v r| < 7.5); e = v r - rne(v r) tells how close it is to a tie,
-// and elements within 1e-5 of one take the IEEE division.  The result needs
-// no clamp (|v r| < 7.5); its low nibble is the two's-complement code.
-__device__ __forceinline__ uint32_t int4_nibble_r(float v, float s, float r) {
-  constexpr float MAGIC = 12582912.0f;   // 1.5 * 2^23
-  if (r == 0.0f) return (uint32_t)int4_code(v, s) & 0xFu;
-  const float t = __fmaf_rn(v, r, MAGIC);
-  const float e = __fmaf_rn(v, r, -__fsub_rn(t, MAGIC));
-  if (fabsf(e) > 0.49999f) return (uint32_t)int4_code(v, s) & 0xFu;
-  return __float_as_uint(t) & 0xFu;
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+
+// Two fp32 products / sums / differences in one instruction, each rounded
+// to nearest on its own (bit-identical to two scalar operations).
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// max(a, |b|, |c|) in one three-input instruction
+__device__ __forceinline__ float max_abs3(float a, float b, float c) {
+  float d;
+  asm("{\n\t.reg .f32 ab, ac;\n\tabs.f32 ab, %2;\n\tabs.f32 ac, %3;\n\tmax.f32 %0, %1, ab, ac;\n\t}"
+      : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+// int4_code(v[e], s[e]) of eight elements without a division per element,
+// for |v| <= 7 s (1 + 2^-22) (every element whose amax gave s = fl(amax / 7)),
+// as the low byte of t[e] (two's complement; the low nibble is the packed
+// code).  With r = RN(1 / s), |v r - v / s| <= |v| 2^-24 / s <= 7.0 * 2^-24
+// and |fl(v / s) - v / s| <= 2^-22, so v r is within 6.6e-7 of fl(v / s):
+// the two round to the same integer unless v r lies within that of a
+// half-integer.  t = v r + 1.5 * 2^23 rounded once is that integer in the low
+// mantissa bits (exact: |v r| < 7.5, so no clamp is needed), and
+// d = v r - (t - 1.5 * 2^23) tells how close it is to a tie.  If any of the
+// eight lies within 1e-5 of a tie, or a scale has no usable reciprocal
+// (no_recip), all eight take the IEEE quotient instead.
+__device__ __forceinline__ void int4_codes8(const float (&v)[8], const float (&s)[8], const float (&r)[8],
+                                            bool no_recip, uint32_t (&t)[8]) {
+  float near = no_recip ? 1.0f : 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float t0, t1, u0, u1, d0, d1;
+    fma2(t0, t1, v[e], v[e + 1], r[e], r[e + 1], kMagic, kMagic);
+    sub2(u0, u1, kMagic, kMagic, t0, t1);
+    fma2(d0, d1, v[e], v[e + 1], r[e], r[e + 1], u0, u1);
+    near = max_abs3(near, d0, d1);
+    t[e] = __float_as_uint(t0);
+    t[e + 1] = __float_as_uint(t1);
+  }
+  if (near > 0.49999f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = (uint32_t)int4_code(v[e], s[e]);
+  }
+}
 
 // Eight codes held in the low bytes of w[0..7] (two's complement) -> one
 // word of nibbles, code e in bits 4e .. 4e + 3: the even codes and the odd
@@ -149,8 +181,11 @@ __device__ __forceinline__ void rope8(const PairTab& pt, const float4* __restric
     const float4 t = in_bounds(ti >= 0 && ti < n_tab, err, 0x101) ? __ldg(&tab[ti]) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
     if (FORM == 1) {          // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
-      y[2 * pp] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
-      y[2 * pp + 1] = __fsub_rn(__fmul_rn(t.w, x0), __fmul_rn(t.z, x1));
+      float p0, p1, q0, q1;
+      mul2(p0, p1, t.z, t.w, x0, x0);
+      mul2(q0, q1, t.w, t.z, x1, x1);
+      y[2 * pp] = __fadd_rn(p0, q0);
+      y[2 * pp + 1] = __fsub_rn(p1, q1);
     } else if (FORM == 2) {   // z0 = m00 x0 + m01 x1, z1 = m10 x0 + m11 x1
       y[2 * pp] = __fadd_rn(__fmul_rn(t.x, x0), __fmul_rn(t.y, x1));
       y[2 * pp + 1] = __fadd_rn(__fmul_rn(t.z, x0), __fmul_rn(t.w, x1));
@@ -315,29 +350,22 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(z[i][e]));
+    for (int e = 0; e < 8; e += 2) amax = max_abs3(amax, z[i][e], z[i][e + 1]);
   amax = block_max(amax, red);
   const float s = __fdiv_rn(amax, 7.0f);
   const float rs = code_recip(s);
-  // codes as in int4_nibble_r, with the closeness to a tie tracked per row
-  // instead of a branch per element: t = z r + 1.5 * 2^23 holds the code in
-  // its low byte (two's complement); a row with any element within 1e-5 of a
-  // tie (or a scale without a usable reciprocal) is redone with the IEEE
-  // quotient
+  // codes of each row: one IEEE division per block for the scale and its
+  // reciprocal, none per element (int4_codes8)
+  float s8[8], r8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    s8[e] = s;
+    r8[e] = rs;
+  }
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     uint32_t tb[8];
-    float near = rs == 0.0f ? 1.0f : 0.0f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float t = __fmaf_rn(z[i][e], rs, kMagic);
-      near = fmaxf(near, fabsf(__fmaf_rn(z[i][e], rs, -__fsub_rn(t, kMagic))));
-      tb[e] = __float_as_uint(t);
-    }
-    if (near > 0.49999f) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) tb[e] = (uint32_t)int4_code(z[i][e], s);
-    }
+    int4_codes8(z[i], s8, r8, rs == 0.0f, tb);
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
     if (in_bounds(n < P.N_pad && bh < P.BH, err, 0x105))
       *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = pack8_low_nibbles(tb);
@@ -384,29 +412,70 @@ __global__ void __launch_bounds__(128) v_amax_kernel(Prob P, const __half* __res
   if (in_bounds(bh < P.BH, err, 0x202)) atomicMax(&vamax[(size_t)bh * D + c], __float_as_uint(r));
 }
 
+// 8 x 8 transpose of nibbles: on entry r[i] holds nibble e of row i in bits
+// 4e .. 4e + 3; on return r[e] holds nibble i of the old r[i] in bits 4i ..
+// 4i + 3.  Three block swaps: 4 x 4 blocks (16-bit halves), 2 x 2 blocks
+// (bytes), single nibbles.
+__device__ __forceinline__ void transpose8_nibbles(uint32_t (&r)[8]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a = r[i], b = r[i + 4];
+    r[i] = __byte_perm(a, b, 0x5410);
+    r[i + 4] = __byte_perm(a, b, 0x7632);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i += (i & 1) ? 3 : 1) {   // 0, 1, 4, 5
+    const uint32_t a = r[i], b = r[i + 2];
+    r[i] = __byte_perm(a, b, 0x6240);
+    r[i + 2] = __byte_perm(a, b, 0x7351);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const uint32_t a = r[i], b = r[i + 1];
+    r[i] = (a & 0x0F0F0F0Fu) | ((b << 4) & 0xF0F0F0F0u);
+    r[i + 1] = ((a >> 4) & 0x0F0F0F0Fu) | (b & 0xF0F0F0F0u);
+  }
+}
+
+// Sum of the eight signed nibbles (two's complement) of w, plus 64: x ^ 8
+// maps a nibble s in [-8, 7] to s + 8 in [0, 15]; the bytes of the even and
+// of the odd nibbles are summed by dp4a onto acc.
+__device__ __forceinline__ int nibble_sum_plus64(uint32_t w, int acc) {
+  const uint32_t x = w ^ 0x88888888u;
+  acc = __dp4a((int)(x & 0x0F0F0F0Fu), 0x01010101, acc);
+  return __dp4a((int)((x >> 4) & 0x0F0F0F0Fu), 0x01010101, acc);
+}
+
 // One CTA = one 64-token block of V of one head: codes with the per-channel
 // scale, transposed packing (channel-major, two tokens per byte) and the
-// block's column sums.
+// block's column sums.  Thread t holds channels 8 (t % 16) .. + 7 of the 8
+// consecutive tokens 8 (t / 16) .. + 7: it packs each token's 8 codes into a
+// word, transposes the 8 x 8 nibbles in registers (one word per channel, its
+// 8 tokens in order), and the words meet in shared memory, one 32-byte row of
+// 64 tokens per channel.
 __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
                                                       const uint32_t* __restrict__ vamax,
                                                       uint8_t* __restrict__ v4t, float* __restrict__ sv,
                                                       int32_t* __restrict__ vsum,
                                                       const WsHeader* __restrict__ hdr) {
-  __shared__ int8_t codes[QK_BLOCK][D + 16];
+  __shared__ __align__(16) uint32_t words[8][D];   // [token group][channel]
   if (!signature_ok(hdr, P, 0x300)) return;
   DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
   float s[8], rs[8];
+  bool no_recip = false;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
     rs[e] = code_recip(s[e]);
+    no_recip |= rs[e] == 0.0f;
   }
+  uint32_t tw[8];   // token 8 r0 + i: its 8 codes as nibbles
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int n = blk * QK_BLOCK + r0 + 8 * i;
+    const int n = blk * QK_BLOCK + 8 * r0 + i;
     float f[8];
     if (n < P.N && in_bounds(bh < P.BH, err, 0x301)) {
       h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
@@ -415,24 +484,22 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
       for (int e = 0; e < 8; ++e) f[e] = 0.0f;
     }
     if (P.v_rot) hadamard128(f, g);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)   // the nibble, sign-extended
-      codes[r0 + 8 * i][8 * g + e] = (int8_t)((int)(int4_nibble_r(f[e], s[e], rs[e]) << 28) >> 28);
+    uint32_t tb[8];
+    int4_codes8(f, s, rs, no_recip, tb);
+    tw[i] = pack8_low_nibbles(tb);
   }
+  transpose8_nibbles(tw);   // tw[e]: channel 8 g + e, tokens 8 r0 .. 8 r0 + 7
+  uint4* wrow = reinterpret_cast<uint4*>(&words[r0][8 * g]);
+  wrow[0] = make_uint4(tw[0], tw[1], tw[2], tw[3]);
+  wrow[1] = make_uint4(tw[4], tw[5], tw[6], tw[7]);
   __syncthreads();
   const int c = threadIdx.x;
   uint32_t w[8];
-  int sum = 0;
+  int sum = -512;
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int code = codes[8 * t + e][c];
-      sum += code;
-      word |= (uint32_t)(code & 0xF) << (4 * e);
-    }
-    w[t] = word;
+    w[t] = words[t][c];
+    sum = nibble_sum_plus64(w[t], sum);
   }
   // tile-major V^T: [bh][tile][channel][64 bytes], this block is half (blk % 2) of tile blk / 2
   uint4* dst = reinterpret_cast<uint4*>(v4t + (((size_t)bh * (P.N_pad / TILE) + blk / 2) * D + c) * (TILE / 2) +
