@@ -253,7 +253,6 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
   __shared__ float red[QK_THREADS / 32];
   constexpr bool HALF_PAIRS = ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF;
   __shared__ float ys[HALF_PAIRS ? QK_BLOCK : 1][HALF_PAIRS ? D + 4 : 1];
-  if (!signature_ok(hdr, P, 0x100)) return;
   DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
@@ -269,6 +268,8 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
     raw[i] = n < P.N && in_bounds(bh < P.BH, err, 0x102) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0))
                                                          : make_uint4(0, 0, 0, 0);
   }
+  // the data loads above need nothing from the workspace; its tables do
+  if (!signature_ok(hdr, P, 0x100)) return;
   float z[QK_ROWS][8];
   float amax = 0.0f;
   const PairTab pt = pair_tab(P, c0);
@@ -452,37 +453,52 @@ __device__ __forceinline__ int nibble_sum_plus64(uint32_t w, int acc) {
 // consecutive tokens 8 (t / 16) .. + 7: it packs each token's 8 codes into a
 // word, transposes the 8 x 8 nibbles in registers (one word per channel, its
 // 8 tokens in order), and the words meet in shared memory, one 32-byte row of
-// 64 tokens per channel.
-__global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __restrict__ v,
+// 64 tokens per channel.  The 8 row loads are issued first, before the
+// workspace signature is read, and the channel scales are computed once per
+// channel (thread c: channel c) and shared; 8 CTAs per SM (64 registers).
+__global__ void __launch_bounds__(128, 8) v_quant_kernel(Prob P, const __half* __restrict__ v,
                                                       const uint32_t* __restrict__ vamax,
                                                       uint8_t* __restrict__ v4t, float* __restrict__ sv,
                                                       int32_t* __restrict__ vsum,
                                                       const WsHeader* __restrict__ hdr) {
   __shared__ __align__(16) uint32_t words[8][D];   // [token group][channel]
-  if (!signature_ok(hdr, P, 0x300)) return;
+  __shared__ __align__(16) float scl[2][D];         // per channel: s, RN(1 / s)
   DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;
   const __half* x = v + (size_t)bh * P.N * D;
-  float s[8], rs[8];
-  bool no_recip = false;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    s[e] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + 8 * g + e]), 7.0f);
-    rs[e] = code_recip(s[e]);
-    no_recip |= rs[e] == 0.0f;
-  }
-  uint32_t tw[8];   // token 8 r0 + i: its 8 codes as nibbles
+  uint4 raw[8];   // token 8 r0 + i, channels 8 g .. 8 g + 7
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int n = blk * QK_BLOCK + 8 * r0 + i;
-    float f[8];
-    if (n < P.N && in_bounds(bh < P.BH, err, 0x301)) {
-      h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g)), f);
-    } else {
+    raw[i] = n < P.N && in_bounds(bh < P.BH, err, 0x301) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + 8 * g))
+                                                         : make_uint4(0, 0, 0, 0);
+  }
+  {   // one division pair per channel: thread c computes channel c's
+    const int c = threadIdx.x;
+    const float sc = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
+    scl[0][c] = sc;
+    scl[1][c] = code_recip(sc);
+    if (!signature_ok(hdr, P, 0x300)) return;
+    if (blk == 0) sv[(size_t)bh * D + c] = sc;
+  }
+  __syncthreads();
+  float s[8], rs[8];
+  {
+    const float4* s4 = reinterpret_cast<const float4*>(&scl[0][8 * g]);
+    const float4* r4 = reinterpret_cast<const float4*>(&scl[1][8 * g]);
+    const float4 sa = s4[0], sb = s4[1], ra = r4[0], rb = r4[1];
+    s[0] = sa.x; s[1] = sa.y; s[2] = sa.z; s[3] = sa.w; s[4] = sb.x; s[5] = sb.y; s[6] = sb.z; s[7] = sb.w;
+    rs[0] = ra.x; rs[1] = ra.y; rs[2] = ra.z; rs[3] = ra.w; rs[4] = rb.x; rs[5] = rb.y; rs[6] = rb.z; rs[7] = rb.w;
+  }
+  bool no_recip = false;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = 0.0f;
-    }
+  for (int e = 0; e < 8; ++e) no_recip |= rs[e] == 0.0f;
+  uint32_t tw[8];   // token 8 r0 + i: its 8 codes as nibbles
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float f[8];
+    h8_to_f(raw[i], f);
     if (P.v_rot) hadamard128(f, g);
     uint32_t tb[8];
     int4_codes8(f, s, rs, no_recip, tb);
@@ -508,7 +524,6 @@ __global__ void __launch_bounds__(128) v_quant_kernel(Prob P, const __half* __re
   dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
   dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
   vsum[((size_t)bh * (P.N_pad / QK_BLOCK) + blk) * D + c] = sum;
-  if (blk == 0) sv[(size_t)bh * D + c] = __fdiv_rn(__uint_as_float(vamax[(size_t)bh * D + c]), 7.0f);
 }
 
 // FP16 path: RoPE of Q and K rounded to fp16 ([BH][N_pad][128], padded rows
