@@ -142,8 +142,9 @@ __device__ __forceinline__ bool signature_ok(const WsHeader* hdr, const Prob& P,
   return false;
 }
 
-// Where the 4 adjacent pairs of channels c0 .. c0 + 7 find their table
-// entries: entry = base[pp] + pos[axis[pp]] * stride[pp].  Computed once per
+// Where a thread's 4 pairs of channels (lo, lo + 1), (lo + 2, lo + 3),
+// (hi, hi + 1), (hi + 2, hi + 3) find their table entries:
+// entry = base[pp] + pos[axis[pp]] * stride[pp].  Computed once per
 // thread with selects on the segment, so that no per-element lookup indexes
 // the problem's arrays with a run-time segment (which would put them in
 // local memory).
@@ -153,11 +154,11 @@ struct PairTab {
 
 __device__ __forceinline__ int sel3(int s, int a, int b, int c) { return s == 0 ? a : (s == 1 ? b : c); }
 
-__device__ __forceinline__ PairTab pair_tab(const Prob& P, int c0) {
+__device__ __forceinline__ PairTab pair_tab(const Prob& P, int lo, int hi) {
   PairTab t;
 #pragma unroll
   for (int pp = 0; pp < 4; ++pp) {
-    const int c = c0 + 2 * pp;
+    const int c = (pp < 2 ? lo : hi) + 2 * (pp & 1);
     const int s = c < P.off[1] ? 0 : (c < P.off[2] ? 1 : 2);
     const int j = (c - sel3(s, P.off[0], P.off[1], P.off[2])) >> 1;
     t.base[pp] = sel3(s, P.tab_off[0], P.tab_off[1], P.tab_off[2]) + j;
@@ -243,16 +244,20 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // One CTA = one 64-token block of Q or K of one head (QK_THREADS threads).
-// Thread t holds channels 8*(t%16) .. +7 of rows (t/16) + QK_RSTEP i.
-template <int ROT>
-__global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF) ? 3 : 4) qk_quant_kernel(Prob P, const __half* __restrict__ q,
+// Thread t holds 8 channels of rows (t/16) + QK_RSTEP i: channels 8 (t%16) ..
+// + 7, or with PAIRS (the Half rotations when every segment and half-segment
+// boundary is a multiple of 4) the 4 channels lo .. lo + 3 of the first half
+// of a segment and their partners lo + d_s/2 .. + 3, so that the rotation
+// needs nothing from other threads.
+template <int ROT, bool PAIRS>
+__global__ void __launch_bounds__(QK_THREADS, ((ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF) && !PAIRS) ? 3 : 4) qk_quant_kernel(Prob P, const __half* __restrict__ q,
                                                        const __half* __restrict__ k, uint8_t* __restrict__ q4,
                                                        uint8_t* __restrict__ k4, float* __restrict__ sq,
                                                        float* __restrict__ sk, const float4* __restrict__ tab,
                                                        const WsHeader* __restrict__ hdr) {
   __shared__ float red[QK_THREADS / 32];
   constexpr bool HALF_PAIRS = ROT == RA_ROT_HALF || ROT == RA_ROT_BLOCKS_HALF;
-  __shared__ float ys[HALF_PAIRS ? QK_BLOCK : 1][HALF_PAIRS ? D + 4 : 1];
+  __shared__ float ys[HALF_PAIRS && !PAIRS ? QK_BLOCK : 1][HALF_PAIRS && !PAIRS ? D + 4 : 1];
   DeviceErr* err = const_cast<DeviceErr*>(&hdr->err);
   const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const __half* x = (which ? k : q) + (size_t)bh * P.N * D;
@@ -260,19 +265,35 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
   float* scale = (which ? sk : sq) + (size_t)bh * (P.N_pad / QK_BLOCK);
   const int g = threadIdx.x & 15, r0 = threadIdx.x >> 4;   // rows r0 + QK_RSTEP i
   const int c0 = 8 * g;
+  int lo = c0, hi = c0 + 4;   // the thread's channels: lo .. lo + 3, hi .. hi + 3
+  int seg = 0;                // PAIRS: the segment of lo and hi
+  if (PAIRS) {
+    // the first half of segment s has split[s] / 8 groups of 4 channels; the
+    // 16 threads of a row take them in order (sum over s: 128 / 8 = 16)
+    const int q0 = P.split[0] >> 3, q1 = P.split[1] >> 3;
+    seg = g < q0 ? 0 : (g < q0 + q1 ? 1 : 2);
+    lo = sel3(seg, P.off[0], P.off[1], P.off[2]) + 4 * (g - sel3(seg, 0, q0, q0 + q1));
+    hi = lo + (sel3(seg, P.split[0], P.split[1], P.split[2]) >> 1);
+  }
 
   uint4 raw[QK_ROWS];
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
-    raw[i] = n < P.N && in_bounds(bh < P.BH, err, 0x102) ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0))
-                                                         : make_uint4(0, 0, 0, 0);
+    const bool ok = n < P.N && in_bounds(bh < P.BH && lo >= 0 && hi + 4 <= D, err, 0x102);
+    if (PAIRS) {
+      const uint2 a = ok ? __ldg(reinterpret_cast<const uint2*>(x + (size_t)n * D + lo)) : make_uint2(0, 0);
+      const uint2 b = ok ? __ldg(reinterpret_cast<const uint2*>(x + (size_t)n * D + hi)) : make_uint2(0, 0);
+      raw[i] = make_uint4(a.x, a.y, b.x, b.y);
+    } else {
+      raw[i] = ok ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
+    }
   }
   // the data loads above need nothing from the workspace; its tables do
   if (!signature_ok(hdr, P, 0x100)) return;
   float z[QK_ROWS][8];
   float amax = 0.0f;
-  const PairTab pt = pair_tab(P, c0);
+  const PairTab pt = pair_tab(P, lo, hi);
 #pragma unroll
   for (int i = 0; i < QK_ROWS; ++i) {
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
@@ -282,7 +303,30 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
     rope8<ROT == RA_ROT_INTERLEAVED ? 1 : (ROT == RA_ROT_BLOCKS_INTERLEAVED ? 2 : 0)>(pt, tab, tp, xf, z[i], P.n_tab,
                                                                                       err);
   }
-  if (HALF_PAIRS) {
+  if (HALF_PAIRS && PAIRS) {
+    // pair (o_s + i, o_s + i + d_s/2) = (z[e], z[4 + e]) of the same thread
+    float4 r4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {   // block of pair o_s / 2 + i, i = index in the first half
+      const int off = sel3(seg, P.off[0], P.off[1], P.off[2]);
+      const int bi = (off >> 1) + (lo + e - off);
+      r4[e] = ROT == RA_ROT_BLOCKS_HALF && in_bounds(bi >= 0 && bi < D / 2, err, 0x107) ? __ldg(&tab[P.n_tab + bi])
+                                                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < QK_ROWS; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = z[i][e], b = z[i][4 + e];
+        if (ROT == RA_ROT_BLOCKS_HALF) {
+          z[i][e] = __fadd_rn(__fmul_rn(r4[e].x, a), __fmul_rn(r4[e].y, b));
+          z[i][4 + e] = __fadd_rn(__fmul_rn(r4[e].z, a), __fmul_rn(r4[e].w, b));
+        } else {
+          z[i][e] = __fmul_rn(__fadd_rn(a, b), kRsqrt2);
+          z[i][4 + e] = __fmul_rn(__fsub_rn(a, b), kRsqrt2);
+        }
+      }
+  } else if (HALF_PAIRS) {
     // pair (o_s + i, o_s + i + d_s/2): each thread has its own channel in a
     // register and reads the partner's value of the same row from shared memory
 #pragma unroll
@@ -299,49 +343,21 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
                      : __fadd_rn(__fmul_rn(r4.z, a), __fmul_rn(r4.w, b));
       return first ? __fmul_rn(__fadd_rn(a, b), kRsqrt2) : __fmul_rn(__fsub_rn(a, b), kRsqrt2);
     };
-    if (P.half4) {
-      // every segment and half-segment boundary is a multiple of 4: a group of
-      // 4 channels shares its segment and half, and its partners are 4
-      // consecutive channels (one 16-byte load)
+    // (the PAIRS instance serves the layouts with every boundary a multiple of 4)
 #pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) {
-        const int c4 = c0 + 4 * q4;
-        const int s = segment_of(P, c4);
-        const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
-        const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
-        const bool first = (c4 - off) < h;
-        const int pc = first ? c4 + h : c4 - h;
-        float4 r4[4];
+    for (int e = 0; e < 8; ++e) {
+      const int c = c0 + e;
+      const int s = segment_of(P, c);
+      const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+      const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
+      const bool first = (c - off) < h;
+      const int pc = first ? c + h : c - h;
+      const float4 r4 = ROT == RA_ROT_BLOCKS_HALF &&
+                                in_bounds((off >> 1) + (c - off) - (first ? 0 : h) < D / 2, err, 0x104)
+                            ? __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)])
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)   // block of pair off_s / 2 + i, i = index in the first half
-          r4[e] = ROT == RA_ROT_BLOCKS_HALF &&
-                          in_bounds((off >> 1) + (c4 + e - off) - (first ? 0 : h) < D / 2, err, 0x103)
-                      ? __ldg(&tab[P.n_tab + (off >> 1) + (c4 + e - off) - (first ? 0 : h)])
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < QK_ROWS; ++i) {
-          const float4 o = *reinterpret_cast<const float4*>(&ys[r0 + QK_RSTEP * i][pc]);
-          const float other[4] = {o.x, o.y, o.z, o.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) z[i][4 * q4 + e] = pair_rot(first, z[i][4 * q4 + e], other[e], r4[e]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int c = c0 + e;
-        const int s = segment_of(P, c);
-        const int h = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
-        const int off = sel3(s, P.off[0], P.off[1], P.off[2]);
-        const bool first = (c - off) < h;
-        const int pc = first ? c + h : c - h;
-        const float4 r4 = ROT == RA_ROT_BLOCKS_HALF &&
-                                  in_bounds((off >> 1) + (c - off) - (first ? 0 : h) < D / 2, err, 0x104)
-                              ? __ldg(&tab[P.n_tab + (off >> 1) + (c - off) - (first ? 0 : h)])
-                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < QK_ROWS; ++i) z[i][e] = pair_rot(first, z[i][e], ys[r0 + QK_RSTEP * i][pc], r4);
-      }
+      for (int i = 0; i < QK_ROWS; ++i) z[i][e] = pair_rot(first, z[i][e], ys[r0 + QK_RSTEP * i][pc], r4);
     }
   }
   if (ROT == RA_ROT_FULL) {
@@ -368,8 +384,15 @@ __global__ void __launch_bounds__(QK_THREADS, (ROT == RA_ROT_HALF || ROT == RA_R
     uint32_t tb[8];
     int4_codes8(z[i], s8, r8, rs == 0.0f, tb);
     const int n = blk * QK_BLOCK + r0 + QK_RSTEP * i;
-    if (in_bounds(n < P.N_pad && bh < P.BH, err, 0x105))
-      *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = pack8_low_nibbles(tb);
+    if (in_bounds(n < P.N_pad && bh < P.BH, err, 0x105)) {
+      const uint32_t w = pack8_low_nibbles(tb);   // codes of lo .. lo + 3 low, hi .. hi + 3 high
+      if (PAIRS) {
+        *reinterpret_cast<uint16_t*>(out + (size_t)n * (D / 2) + lo / 2) = (uint16_t)(w & 0xFFFFu);
+        *reinterpret_cast<uint16_t*>(out + (size_t)n * (D / 2) + hi / 2) = (uint16_t)(w >> 16);
+      } else {
+        *reinterpret_cast<uint32_t*>(out + (size_t)n * (D / 2) + 4 * g) = w;
+      }
+    }
   }
   if (threadIdx.x == 0 && in_bounds(blk < P.N_pad / QK_BLOCK && bh < P.BH, err, 0x106)) scale[blk] = s;
 }
@@ -554,7 +577,7 @@ __global__ void __launch_bounds__(128) fp16_prologue_kernel(Prob P, const __half
       if (n < P.N) {
         float xf[8], y[8];
         h8_to_f(__ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)), xf);
-        rope8<0>(pair_tab(P, c0), tab, token_pos(P, n), xf, y, P.n_tab, err);
+        rope8<0>(pair_tab(P, c0, c0 + 4), tab, token_pos(P, n), xf, y, P.n_tab, err);
         __half2* h = reinterpret_cast<__half2*>(&o);
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
@@ -598,20 +621,22 @@ cudaError_t launch_prologue(const Prob& p, const __half* q, const __half* k, con
   const float4* tab = reinterpret_cast<const float4*>(base + L.tables);
   uint32_t* vamax = reinterpret_cast<uint32_t*>(base + L.vamax);
   const dim3 gqk(p.N_pad / QK_BLOCK, p.BH, 2);
+#define RA_QK(ROT, PAIRS) qk_quant_kernel<ROT, PAIRS><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr)
   switch (p.rot) {
-    case RA_ROT_NONE: qk_quant_kernel<RA_ROT_NONE><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
-    case RA_ROT_INTERLEAVED:
-      qk_quant_kernel<RA_ROT_INTERLEAVED><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
-      break;
-    case RA_ROT_FULL: qk_quant_kernel<RA_ROT_FULL><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
-    case RA_ROT_BLOCKS_INTERLEAVED:
-      qk_quant_kernel<RA_ROT_BLOCKS_INTERLEAVED><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
-      break;
+    case RA_ROT_NONE: RA_QK(RA_ROT_NONE, false); break;
+    case RA_ROT_INTERLEAVED: RA_QK(RA_ROT_INTERLEAVED, false); break;
+    case RA_ROT_FULL: RA_QK(RA_ROT_FULL, false); break;
+    case RA_ROT_BLOCKS_INTERLEAVED: RA_QK(RA_ROT_BLOCKS_INTERLEAVED, false); break;
     case RA_ROT_BLOCKS_HALF:
-      qk_quant_kernel<RA_ROT_BLOCKS_HALF><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr);
+      if (p.half4) RA_QK(RA_ROT_BLOCKS_HALF, true);
+      else RA_QK(RA_ROT_BLOCKS_HALF, false);
       break;
-    default: qk_quant_kernel<RA_ROT_HALF><<<gqk, QK_THREADS, 0, st>>>(p, q, k, q4, k4, sq, sk, tab, hdr); break;
+    default:
+      if (p.half4) RA_QK(RA_ROT_HALF, true);
+      else RA_QK(RA_ROT_HALF, false);
+      break;
   }
+#undef RA_QK
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(vamax, 0, sizeof(uint32_t) * (size_t)p.BH * D, st);
