@@ -399,7 +399,8 @@ def our_arm(args, cfg, rank, world):
                 "h2d_bytes_per_step": 3 * BH * cfg.N * cfg.d * 2, "d2h_bytes_per_step": BH * cfg.N * cfg.d * 2,
                 "api": "ra_int4_attention_host (pinned host q, k, v, o; copies overlapped over head chunks)",
                 "chunks": (f"{args.chunk_heads} heads each" if args.chunk_heads else
-                           f"library default: ramp 1, 2, 3, ... up to {-(-BH // 8)} heads and back down"),
+                           f"library default: ramp 1, 1, 2, 2, ... up to {-(-BH // 8)} heads and back down, three "
+                           f"staging slots"),
                 "serial_ms_per_step": ms_e2e_serial},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),

@@ -200,19 +200,21 @@ size_t ra_host_staging_bytes(const ra_problem *p, int heads_per_chunk);
  * chunks of consecutive heads, each chunk as a problem of its own with B = 1
  * (every step of the path is independent per head, so the results are
  * bit-identical to the device-buffer calls).  heads_per_chunk > 0: chunks of
- * that many heads; 0: chunks of about B*H/8 heads, entered and left by ramps
- * of 1, 2, 3, ... heads, so that the kernels start after a one-head copy and
- * the last copy back is of one head.  While chunk c is computed, the inputs
- * of chunk c+1 are copied in and the output of chunk c-1 is copied out;
- * chunks alternate between `stream` and a second compute stream so that the
- * kernels of chunk c+1 start on the SMs chunk c's last wave leaves idle.  The
- * call creates and destroys its three extra streams and six events.  The
+ * that many heads; 0: chunks of about B*H/8 heads, entered by the ramp 1, 1,
+ * 2, 2, 3, 3, 4, 4, ... and left by ..., 3, 2, 1 heads (ra_host_chunks lists
+ * them), so that the kernels start after a one-head copy and the last copy
+ * back is of one head.  Three staging slots let the inputs of up to two
+ * chunks ahead be copied in while chunk c is computed, and the output of
+ * chunk c-1 is copied out meanwhile; chunks alternate between `stream` and a
+ * second compute stream so that the kernels of chunk c+1 start on the SMs
+ * chunk c's last wave leaves idle.  The call creates and destroys its three
+ * extra streams and eleven events.  The
  * copies overlap only if the host buffers are page-locked (cudaHostAlloc /
  * cudaHostRegister); pageable buffers give the same result without the
  * overlap.
  * staging: device memory owned by the caller, 256-byte aligned, at least
- * ra_host_staging_bytes(p, heads_per_chunk) bytes: two slots, each with q, k,
- * v, o, the quantised tensors and a workspace for the largest chunk.  The
+ * ra_host_staging_bytes(p, heads_per_chunk) bytes: three slots, each with q,
+ * k, v, o, the quantised tensors and a workspace for the largest chunk.  The
  * call blocks until o is written and the device error words are checked,
  * so it returns any status ra_check_device_error can.  The staging buffer
  * must not be used by other work while the call runs. */

@@ -6,16 +6,18 @@
 // B*H heads are cut into chunks of consecutive heads, each a problem of its
 // own with B = 1.  Four streams form a pipeline over the chunks:
 //
-//   copy-in stream   : q, k, v of chunk c, host -> slot c % 2
-//   compute lane c%2 : prologue + INT4 attention of chunk c (slot c % 2);
+//   copy-in stream   : q, k, v of chunk c, host -> slot c % 3
+//   compute lane c%2 : prologue + INT4 attention of chunk c (slot c % 3);
 //                      lane 0 is the caller's stream, lane 1 one of ours
-//   copy-out stream  : o of chunk c, slot c % 2 -> host
+//   copy-out stream  : o of chunk c, slot c % 3 -> host
 //
 // so that the host->device copy of chunk c+1 and the device->host copy of
 // chunk c-1 run on the copy engines while chunk c is computed, and the
 // kernels of chunk c+1 fill the SMs that the last wave of chunk c leaves idle
 // (each slot has its own quantised tensors and workspace).  Events order the
-// reuse of the two slots.  The call blocks until o is written.
+// reuse of the three slots: the copy-in of chunk c may start once chunk c - 3
+// has been computed, so it runs up to two chunks ahead of the kernels.  The
+// call blocks until o is written.
 #include <algorithm>
 #include <cstdio>
 #include <vector>
@@ -27,6 +29,7 @@
 namespace {
 
 constexpr int kDefaultChunks = 8;   // chunks of the largest size when the caller passes 0
+constexpr int kSlots = 3;           // staging slots: chunk c uses slot c % kSlots
 
 struct HostPlan {
   std::vector<int> heads;     // heads of every chunk, in order
@@ -38,11 +41,15 @@ struct HostPlan {
 };
 
 // Chunk sizes.  Given heads_per_chunk > 0: equal chunks (the last one takes
-// the remainder).  Given 0: chunks of about B*H/8 heads, entered and left by
-// ramps 1, 2, 3, ... so that the first kernels wait only for a one-head copy
-// and the last copy-out is of one head (a head's copy-in takes about 3/4 of
-// its compute, so each chunk's copy-in hides behind the previous chunk's
-// kernels when sizes grow by at most 4/3).
+// the remainder).  Given 0: chunks of about B*H/8 heads, entered by the ramp
+// 1, 1, 2, 2, 3, 3, 4, 4, ... and left by ..., 3, 2, 1, so that the first
+// kernels wait only for a one-head copy and the last copy-out is of one
+// head.  A head's copy-in takes about 0.85 of its compute; with three slots
+// the copy-in of chunk c may start once chunk c - 3 has been computed, and
+// each size taken twice on the way up keeps every copy-in behind the
+// kernels of the chunks before it.
+int grow(int k) { return std::max(k + 1, (4 * k) / 3); }
+
 void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
   out.clear();
   if (heads_per_chunk > 0) {
@@ -50,33 +57,35 @@ void chunk_sizes(int BH, int heads_per_chunk, std::vector<int>& out) {
     return;
   }
   const int per = (BH + kDefaultChunks - 1) / kDefaultChunks;
-  std::vector<int> ramp;
-  int ramp_sum = 0;
-  for (int next = 1; next < per; next = std::max(next + 1, (4 * next) / 3)) {
-    ramp.push_back(next);
-    ramp_sum += next;
+  // up: 1, 1, 2, 2, 3, 3, 4, 4, then growing by grow(); down: the plain
+  // grow() ramp, reversed
+  std::vector<int> up, down;
+  for (int k = 1; k < per; k = grow(k)) {
+    up.push_back(k);
+    if (k <= 4) up.push_back(k);
   }
-  if (2 * ramp_sum > BH) {   // too few heads for both ramps: ramp up only
-    int done = 0, next = 1;
-    while (done < BH) {
-      const int c = std::min(std::min(next, per), BH - done);
-      out.push_back(c);
-      done += c;
-      next = std::max(next + 1, (4 * c) / 3);
-    }
-    return;
+  for (int k = 1; k < per; k = grow(k)) down.insert(down.begin(), k);
+  auto sum = [](const std::vector<int>& v) {
+    int t = 0;
+    for (int x : v) t += x;
+    return t;
+  };
+  // the middle: chunks between the ramps' top size and min(per, grow(top));
+  // hand the top steps of both ramps to it until such chunks fit
+  int mid = 0, n_mid = 0;
+  while (true) {
+    const int top = std::max(up.empty() ? 0 : up.back(), down.empty() ? 0 : down.front());
+    const int cap = top ? std::min(per, grow(top)) : per;
+    mid = BH - sum(up) - sum(down);
+    n_mid = (mid + cap - 1) / cap;
+    if (mid >= std::max(top, 1) && mid / n_mid >= top) break;
+    if (up.empty() && down.empty()) break;
+    while (!up.empty() && up.back() >= top) up.pop_back();
+    while (!down.empty() && down.front() >= top) down.erase(down.begin());
   }
-  // the middle (chunks of at most per heads, balanced) must not dip below the
-  // ramp's top: hand the top steps of both ramps to the middle until it fits
-  int mid = BH - 2 * ramp_sum;
-  while (!ramp.empty() && mid < ramp.back()) {
-    mid += 2 * ramp.back();
-    ramp.pop_back();
-  }
-  out = ramp;
-  const int n_mid = (mid + per - 1) / per;
+  out = up;
   for (int i = 0; i < n_mid; ++i) out.push_back(mid / n_mid + (i < mid % n_mid ? 1 : 0));
-  out.insert(out.end(), ramp.rbegin(), ramp.rend());
+  out.insert(out.end(), down.begin(), down.end());
 }
 
 ra_status plan(const ra_problem* p, int heads_per_chunk, HostPlan* hp) {
@@ -99,7 +108,7 @@ ra_status plan(const ra_problem* p, int heads_per_chunk, HostPlan* hp) {
   h.qkv4 = ra::align256(ra_qkv4_bytes(&h.chunk));
   h.io = ra::align256(4 * h.per * h.head_bytes);    // q, k, v, o of one chunk
   h.slot = h.ws + h.qkv4 + h.io;
-  h.total = 2 * h.slot;
+  h.total = kSlots * h.slot;
   return RA_OK;
 }
 
@@ -114,9 +123,12 @@ ra_status cuda_err(cudaError_t e, const char* what) {
 // Streams and events of one call, released on every path out of it.
 struct Pipeline {
   cudaStream_t in = nullptr, out = nullptr, lane1 = nullptr;
-  cudaEvent_t loaded[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr}, stored[2] = {nullptr, nullptr};
+  cudaEvent_t loaded[kSlots] = {}, computed[kSlots] = {}, stored[kSlots] = {};
+  cudaEvent_t lane_done[2] = {};
   ~Pipeline() {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2; ++i)
+      if (lane_done[i]) cudaEventDestroy(lane_done[i]);
+    for (int i = 0; i < kSlots; ++i) {
       if (loaded[i]) cudaEventDestroy(loaded[i]);
       if (computed[i]) cudaEventDestroy(computed[i]);
       if (stored[i]) cudaEventDestroy(stored[i]);
@@ -129,7 +141,8 @@ struct Pipeline {
     cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&lane1, cudaStreamNonBlocking);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&lane_done[i], cudaEventDisableTiming);
+    for (int i = 0; i < kSlots && e == cudaSuccess; ++i) {
       e = cudaEventCreateWithFlags(&loaded[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&computed[i], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&stored[i], cudaEventDisableTiming);
@@ -177,11 +190,12 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(staging);
-  void* ws[2] = {base, base + h.slot};
+  void* ws[kSlots];
+  for (int i = 0; i < kSlots; ++i) ws[i] = base + i * h.slot;
 
-  // Tables and signature of both slots' workspaces (synchronises `stream`);
+  // Tables and signature of every slot's workspace (synchronises `stream`);
   // the signature does not cover B or H, so each serves every chunk size.
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < kSlots; ++i)
     if ((st = ra_prepare(&h.chunk, ws[i], h.ws, stream)) != RA_OK) return st;
 
   Pipeline pl;
@@ -195,7 +209,7 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   char* oh = static_cast<char*>(o);
   size_t off = 0;   // first byte of the chunk in every host tensor
   for (size_t c = 0; c < h.heads.size(); ++c) {
-    const int sl = (int)(c & 1);
+    const int sl = (int)(c % kSlots), ln = (int)(c & 1);
     ra_problem cp = h.chunk;
     cp.H = h.heads[c];
     char* slot = base + sl * h.slot;
@@ -205,20 +219,20 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
     char* io = slot + h.ws + h.qkv4;
     char *qd = io, *kd = io + n, *vd = io + 2 * n, *od = io + 3 * n;
 
-    // copy-in: the slot is free once chunk c-2 has been computed
-    if (c >= 2 && (e = cudaStreamWaitEvent(pl.in, pl.computed[sl], 0)) != cudaSuccess) break;
+    // copy-in: the slot is free once chunk c - kSlots has been computed
+    if (c >= (size_t)kSlots && (e = cudaStreamWaitEvent(pl.in, pl.computed[sl], 0)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(qd, qh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(kd, kh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaMemcpyAsync(vd, vh + off, n, cudaMemcpyHostToDevice, pl.in)) != cudaSuccess) break;
     if ((e = cudaEventRecord(pl.loaded[sl], pl.in)) != cudaSuccess) break;
 
     // compute on lane c % 2 (after chunk c-2 on the same lane): inputs
-    // loaded, and the slot's output read back (chunk c-2)
-    if ((e = cudaStreamWaitEvent(lane[sl], pl.loaded[sl], 0)) != cudaSuccess) break;
-    if (c >= 2 && (e = cudaStreamWaitEvent(lane[sl], pl.stored[sl], 0)) != cudaSuccess) break;
-    if ((st = ra_rotate_quantize_qkv(&cp, qd, kd, vd, &qkv, ws[sl], h.ws, lane[sl])) != RA_OK) break;
-    if ((st = ra_int4_attention_fwd(&cp, &qkv, od, ws[sl], h.ws, lane[sl])) != RA_OK) break;
-    if ((e = cudaEventRecord(pl.computed[sl], lane[sl])) != cudaSuccess) break;
+    // loaded, and the slot's output read back (chunk c - kSlots)
+    if ((e = cudaStreamWaitEvent(lane[ln], pl.loaded[sl], 0)) != cudaSuccess) break;
+    if (c >= (size_t)kSlots && (e = cudaStreamWaitEvent(lane[ln], pl.stored[sl], 0)) != cudaSuccess) break;
+    if ((st = ra_rotate_quantize_qkv(&cp, qd, kd, vd, &qkv, ws[sl], h.ws, lane[ln])) != RA_OK) break;
+    if ((st = ra_int4_attention_fwd(&cp, &qkv, od, ws[sl], h.ws, lane[ln])) != RA_OK) break;
+    if ((e = cudaEventRecord(pl.computed[sl], lane[ln])) != cudaSuccess) break;
 
     // copy-out
     if ((e = cudaStreamWaitEvent(pl.out, pl.computed[sl], 0)) != cudaSuccess) break;
@@ -230,8 +244,8 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   // also on an error path (nothing may still use the staging buffer on return).
   cudaError_t j = cudaEventRecord(pl.loaded[0], pl.in);
   if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.loaded[0], 0);
-  if (j == cudaSuccess) j = cudaEventRecord(pl.computed[1], pl.lane1);
-  if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.computed[1], 0);
+  if (j == cudaSuccess) j = cudaEventRecord(pl.lane_done[1], pl.lane1);
+  if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.lane_done[1], 0);
   if (j == cudaSuccess) j = cudaEventRecord(pl.stored[0], pl.out);
   if (j == cudaSuccess) j = cudaStreamWaitEvent(s, pl.stored[0], 0);
   cudaError_t w = cudaStreamSynchronize(s);
@@ -239,8 +253,9 @@ ra_status ra_int4_attention_host(const ra_problem* p, const void* q, const void*
   if (e != cudaSuccess) return cuda_err(e, "pipeline enqueue");
   if (j != cudaSuccess) return cuda_err(j, "pipeline join");
   if (w != cudaSuccess) return cuda_err(w, "pipeline synchronize");
-  if ((st = ra_check_device_error(ws[0], stream)) != RA_OK) return st;
-  return ra_check_device_error(ws[1], stream);
+  for (int i = 0; i < kSlots; ++i)
+    if ((st = ra_check_device_error(ws[i], stream)) != RA_OK) return st;
+  return RA_OK;
 }
 
 }  // extern "C"
