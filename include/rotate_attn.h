@@ -277,7 +277,10 @@ ra_status ra_noalloc_check_device_error(ra_stream stream);
 /* Number of floats of the coefficient table and the table itself, as
  * ra_prepare uploads it: for segment s, position pos in [0, P_s) with
  * P = (F, Hh, W), pair j: {cos, sin, alpha, beta} at
- * 4 * (off_s + pos * split[s]/2 + j), off_0 = 0, off_{s+1} = off_s + P_s*split[s]/2. */
+ * 4 * (off_s + pos * 4 q_s + (j % 4) q_s + j / 4), q_s = ceil(split[s] / 8),
+ * off_0 = 0, off_{s+1} = off_s + P_s * 4 q_s (the other slots of a block are
+ * zero); then the d/2 pair blocks (r00, r01, r10, r11), zero unless the
+ * rotation takes caller blocks. */
 size_t ra_tables_floats(const ra_problem *p);
 ra_status ra_build_tables_host(const ra_problem *p, float *out, size_t n_floats);
 

@@ -4,6 +4,7 @@
 // is the caller's.
 #include <atomic>
 #include <cstdarg>
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -107,7 +108,8 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
       off += p->split[s];
       P.npos[s] = npos[s];
       P.tab_off[s] = toff;
-      toff += npos[s] * (p->split[s] / 2);
+      P.tab_q[s] = (p->split[s] / 2 + 3) / 4;
+      toff += npos[s] * 4 * P.tab_q[s];
     }
     P.fastdiv = 1;
     const uint64_t divs[2] = {(uint64_t)(p->W > 0 ? p->W : 1), (uint64_t)(p->W > 0 ? p->W : 1) * (p->Hh > 0 ? p->Hh : 1)};
@@ -139,9 +141,13 @@ ra_status derive(const ra_problem* p, ra::Prob* out) {
 
 // Coefficients {cos a, sin a, (cos a + sin a)/sqrt2, (cos a - sin a)/sqrt2}
 // per (segment, position, pair), a = pos * theta^(-2j/d_s), each computed in
-// float64 and rounded once to fp32.
+// float64 and rounded once to fp32.  A position's block of segment s has
+// 4 q slots (q = ceil(d_s / 8)), pair j at slot (j % 4) q + j / 4, the rest
+// zero: the 16 threads of a row hold pairs 4g .. 4g + 3 (channels 8g .. 8g +
+// 7), so for each of their four pairs they read consecutive slots.
 void build_tables(const ra_problem* p, const ra::Prob& P, float* out) {
   const bool blocks_mode = p->rot == RA_ROT_BLOCKS_INTERLEAVED || p->rot == RA_ROT_BLOCKS_HALF;
+  std::fill(out, out + 4 * (size_t)P.n_tab, 0.0f);   // the unused slots of each block
   for (int s = 0; s < 3; ++s) {
     const int half = p->split[s] / 2;
     for (int pos = 0; pos < P.npos[s]; ++pos)
@@ -149,7 +155,8 @@ void build_tables(const ra_problem* p, const ra::Prob& P, float* out) {
         const double w = std::pow(p->theta, -(double)(2 * j) / (double)p->split[s]);
         const double a = (double)pos * w;
         const double ca = std::cos(a), sa = std::sin(a);
-        float* e = out + 4 * ((size_t)P.tab_off[s] + (size_t)pos * half + j);
+        const int q = P.tab_q[s];
+        float* e = out + 4 * ((size_t)P.tab_off[s] + (size_t)pos * 4 * q + (size_t)(j % 4) * q + j / 4);
         if (p->rot == RA_ROT_BLOCKS_INTERLEAVED) {   // R times the RoPE rotation, per (pos, pair)
           const double* r = p->blocks + 4 * (P.off[s] / 2 + j);
           e[0] = (float)(r[0] * ca + r[1] * sa);

@@ -23,6 +23,8 @@ struct Prob {
   int split[3], off[3];         // segment sizes and first channel of each segment
   int npos[3];                  // positions per axis: F, Hh, W
   int tab_off[3];               // first table entry of each segment
+  int tab_q[3];                 // ceil(split[s] / 8): a position's block of segment s holds 4 tab_q
+                                // entries, pair j at slot (j % 4) tab_q + j / 4
   int n_tab;                    // RoPE table entries (each: cos, sin, alpha, beta, or for
                                 // BLOCKS_INTERLEAVED the merged m00, m01, m10, m11)
   int n_tab_all;                // n_tab + d/2 pair-block entries (r00, r01, r10, r11)

@@ -161,8 +161,9 @@ __device__ __forceinline__ PairTab pair_tab(const Prob& P, int lo, int hi) {
     const int c = (pp < 2 ? lo : hi) + 2 * (pp & 1);
     const int s = c < P.off[1] ? 0 : (c < P.off[2] ? 1 : 2);
     const int j = (c - sel3(s, P.off[0], P.off[1], P.off[2])) >> 1;
-    t.base[pp] = sel3(s, P.tab_off[0], P.tab_off[1], P.tab_off[2]) + j;
-    t.stride[pp] = sel3(s, P.split[0], P.split[1], P.split[2]) >> 1;
+    const int q = sel3(s, P.tab_q[0], P.tab_q[1], P.tab_q[2]);
+    t.base[pp] = sel3(s, P.tab_off[0], P.tab_off[1], P.tab_off[2]) + (j & 3) * q + (j >> 2);
+    t.stride[pp] = 4 * q;
     t.axis[pp] = s;
   }
   return t;

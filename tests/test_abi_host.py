@@ -211,6 +211,12 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
     rng = np.random.default_rng(0)
     for s in range(3):
         half = cfg.split[s] // 2
+        q = (half + 3) // 4      # a position's block: 4 q slots, pair j at (j % 4) q + j // 4
+        used = np.zeros(4 * q, bool)
+        used[[(j % 4) * q + j // 4 for j in range(half)]] = True
+        assert used.sum() == half                      # distinct slots
+        blocks = tab[k:k + npos[s] * 4 * q].reshape(npos[s], 4 * q, 4)
+        assert not blocks[:, ~used].any()              # the other slots are zero
         # every entry for small grids, a sample for the large ones
         cells = [(pos, j) for pos in range(npos[s]) for j in range(half)]
         if len(cells) > 400:
@@ -218,8 +224,8 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
             cells = [cells[i] for i in idx] + [(npos[s] - 1, half - 1)]
         for pos, j in cells:
             ref = np.array(oracle_mod.rope_coef(cfg, s, pos, j), np.float32)
-            got = tab[k + pos * half + j]
+            got = tab[k + pos * 4 * q + (j % 4) * q + j // 4]
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), (name, s, pos, j)
-        k += npos[s] * half
+        k += npos[s] * 4 * q
     assert k + 64 == len(tab)                 # then the 64 pair-block entries (zero here)
     assert not tab[k:].any()
