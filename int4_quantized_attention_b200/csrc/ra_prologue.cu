@@ -180,7 +180,15 @@ __device__ __forceinline__ void rope8(const PairTab& pt, const float4* __restric
   for (int pp = 0; pp < 4; ++pp) {
     const int pos = sel3(pt.axis[pp], tp.p[0], tp.p[1], tp.p[2]);
     const int ti = pt.base[pp] + pos * pt.stride[pp];
-    const float4 t = in_bounds(ti >= 0 && ti < n_tab, err, 0x101) ? __ldg(&tab[ti]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (in_bounds(ti >= 0 && ti < n_tab, err, 0x101)) {
+      if (FORM == 2) {
+        t = __ldg(&tab[ti]);
+      } else {   // FORM 0 reads (cos, sin), FORM 1 (alpha, beta): one 8-byte load
+        const float2 h = __ldg(reinterpret_cast<const float2*>(&tab[ti]) + (FORM == 1 ? 1 : 0));
+        if (FORM == 1) { t.z = h.x; t.w = h.y; } else { t.x = h.x; t.y = h.y; }
+      }
+    }
     const float x0 = x[2 * pp], x1 = x[2 * pp + 1];
     if (FORM == 1) {          // z0 = alpha x0 + beta x1, z1 = beta x0 - alpha x1
       float p0, p1, q0, q1;
@@ -290,8 +298,6 @@ __global__ void __launch_bounds__(QK_THREADS, ((ROT == RA_ROT_HALF || ROT == RA_
       raw[i] = ok ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)n * D + c0)) : make_uint4(0, 0, 0, 0);
     }
   }
-  // the data loads above need nothing from the workspace; its tables do
-  if (!signature_ok(hdr, P, 0x100)) return;
   float z[QK_ROWS][8];
   float amax = 0.0f;
   const PairTab pt = pair_tab(P, lo, hi);
@@ -370,6 +376,9 @@ __global__ void __launch_bounds__(QK_THREADS, ((ROT == RA_ROT_HALF || ROT == RA_
 #pragma unroll
     for (int e = 0; e < 8; e += 2) amax = max_abs3(amax, z[i][e], z[i][e + 1]);
   amax = block_max(amax, red);
+  // the workspace's tables were read above (in bounds whatever they hold);
+  // nothing is written unless they are this problem's
+  if (!signature_ok(hdr, P, 0x100)) return;
   const float s = __fdiv_rn(amax, 7.0f);
   const float rs = code_recip(s);
   // codes of each row: one IEEE division per block for the scale and its
