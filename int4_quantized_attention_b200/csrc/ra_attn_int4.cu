@@ -555,11 +555,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
       auto wait = [&](int b, uint32_t parity, uint32_t site) {
         return mbar_spin_abortable(&bar[b], parity, abort_flag, limit, err, site);
       };
+      // A 32-byte step along K adds 2 to a descriptor's address field
+      // (address / 16 in bits 0-13; every operand lies below 2^18 bytes and
+      // starts on a 1024-byte boundary, so the field never carries).
+      const uint64_t dq = sw128_desc(qa);
       auto issue_S = [&](int j) {   // S_X(j) = 256 Q_X K(j)^T
-        const uint32_t kt = op + (j % OP_STAGES) * 32768;
+        const uint64_t dk = sw128_desc(op + (j % OP_STAGES) * 32768);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_i8(tS, sw128_desc(qa + 32 * kk), sw128_desc(kt + 32 * kk), IDESC_QK, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) umma_i8(tS, dq + 2 * kk, dk + 2 * kk, IDESC_QK, kk > 0);
         umma_commit(&bar[B_S_FULL + X]);
       };
       bool ok = wait(B_QFULL, 0, 0x4301) && wait(B_OP_FULL, 0, 0x4302);
@@ -576,11 +579,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) int4_attn_kernel(const KernelA
         }
         if (!(ok = wait(B_P_FULL + 2 * X + (j & 1), (j >> 1) & 1, 0x4305))) break;
         tc_fence_after();
-        const uint32_t vt = op + (j % OP_STAGES) * 32768 + 16384;   // O_X += W_X(j) V(j)
-        const uint32_t pa = pbase + (j & 1) * 16384;
+        const uint64_t dv = sw128_desc(op + (j % OP_STAGES) * 32768 + 16384);   // O_X += W_X(j) V(j)
+        const uint64_t dp = sw128_desc(pbase + (j & 1) * 16384);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_i8(tO, sw128_desc(pa + 32 * kk), sw128_desc(vt + 32 * kk), IDESC_PV, 1);   // onto MB
+        for (int kk = 0; kk < 4; ++kk) umma_i8(tO, dp + 2 * kk, dv + 2 * kk, IDESC_PV, 1);   // onto MB
         umma_commit(&bar[B_PV_DONE + 2 * X + (j & 1)]);
         umma_commit(&bar[B_OP_EMPTY + j % OP_STAGES]);
       }
