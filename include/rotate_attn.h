@@ -245,7 +245,9 @@ const char *ra_last_error_detail(void);
  * -- lives in one fixed array of RA_NOALLOC_SCRATCH_BYTES inside this
  * library, which every GPU that loads the library holds until the process
  * exits.  Problems whose scratch would not fit (about 512 bytes per head plus
- * 16 bytes per RoPE table entry, plus a 256-byte header) are rejected with
+ * 16 bytes per RoPE table slot -- 4 ceil(split[s] / 8) slots per position of
+ * segment s -- plus 16 bytes per channel pair and a 256-byte header) are
+ * rejected with
  * RA_ERR_WORKSPACE before anything is enqueued.  The call allocates nothing
  * (no cudaMalloc, cudaFree or allocating library routine); it copies the
  * tables from static host memory with cudaMemcpyAsync on `stream` (a pageable
