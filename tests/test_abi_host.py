@@ -229,3 +229,17 @@ def test_tables_bit_exact_against_oracle(lib, oracle_mod, name):
         k += npos[s] * 4 * q
     assert k + 64 == len(tab)                 # then the 64 pair-block entries (zero here)
     assert not tab[k:].any()
+
+
+def test_host_chunk_schedule_every_head_count(lib):
+    """The default schedule's invariants for every B*H up to 2000: it covers
+    the heads, stays within ceil(B*H/8) heads a chunk, starts with one head
+    (and ends with one when there are at least 8), and grows by at most 4/3
+    (+1) per step."""
+    for BH in range(1, 2001):
+        p = api.problem(synth.CONFIGS["tiny"].replace(B=1, H=BH))
+        per = -(-BH // 8)
+        c = api.host_chunks(p, 0)
+        assert sum(c) == BH and min(c) >= 1 and max(c) <= per and c[0] == 1, BH
+        assert all(b <= max(a + 1, 4 * a // 3) for a, b in zip(c, c[1:])), (BH, c)
+        assert BH < 8 or c[-1] == 1, (BH, c)
